@@ -1,0 +1,125 @@
+"""Seeded synthetic MLA-decode workloads (shapes, lengths, values).
+
+This module only draws random inputs; it holds none of the attention
+arithmetic, so both the CUDA path's tests and the fp64 oracle can use it
+without sharing any of the method's code.
+
+Recipe (identical on every machine, CPU generators only):
+  * lengths: fixed per workload, or for the mixed-length workload
+    ``torch.randint(lo, hi + 1, (B,))`` from ``torch.Generator().manual_seed(seed)``;
+  * per sequence b, q[b] is ``torch.randn(Sq, H, 576) * sigma`` and the first
+    L_b rows of kv[b] are ``torch.randn(L_b, 576) * sigma``, each from its own
+    generator seeded with ``_stream_seed(seed, b, which)``, then rounded to
+    bfloat16 (round to nearest even);
+  * kv rows L_b .. L_max-1 are filled with ``tail_fill`` (NaN in the parity
+    tests, so any read past a sequence's end shows up in the result).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import torch
+
+D_QK = 576      # 512 latent + 64 rope columns per cached row
+D_V = 512       # values are the first 512 columns of the same rows
+D_ROPE = 64
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Sq: int
+    H: int
+    L: int                      # L_max (every sequence has this length unless L_lo is set)
+    L_lo: Optional[int] = None  # mixed lengths: uniform integers in [L_lo, L]
+    sigma: float = 1.0
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        # softmax scale 576^-0.5 (= 1/24 in real arithmetic), as an fp32 value
+        return float(torch.tensor(D_QK ** -0.5, dtype=torch.float32).item())
+
+    def lengths(self) -> torch.Tensor:
+        if self.L_lo is None:
+            return torch.full((self.B,), self.L, dtype=torch.int32)
+        g = torch.Generator().manual_seed(self.seed)
+        return torch.randint(self.L_lo, self.L + 1, (self.B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+    def algorithmic_bytes(self, lengths: Optional[torch.Tensor] = None) -> int:
+        """Bytes a perfect kernel must move: each used kv row once (V aliases
+        K), q, out (bf16), lse (fp32) and the lengths array."""
+        sl = self.lengths() if lengths is None else lengths
+        rows = self.B * self.Sq * self.H
+        return int(sl.to(torch.int64).sum()) * D_QK * 2 + rows * (D_QK * 2 + D_V * 2 + 4) + self.B * 4
+
+    def algorithmic_flops(self, lengths: Optional[torch.Tensor] = None) -> int:
+        """2*(576+512) flops per (query row, key): QK^T and PV, exps not counted."""
+        sl = self.lengths() if lengths is None else lengths
+        return int(sl.to(torch.int64).sum()) * self.Sq * self.H * 2 * (D_QK + D_V)
+
+
+# The five parity/benchmark workloads, plus the headline-metric line
+# (mixed-length workload's shape with every sequence at L = 8192).
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, Sq=1, H=16, L=256, seed=1000),
+    "dsv3": Workload("dsv3", B=16, Sq=1, H=128, L=4096, seed=1001),
+    "mixed": Workload("mixed", B=64, Sq=1, H=128, L=8192, L_lo=1024, seed=1002),
+    "lowhead": Workload("lowhead", B=132, Sq=1, H=16, L=16384, seed=1003),
+    "long": Workload("long", B=4, Sq=2, H=128, L=131072, sigma=0.5, seed=1004),
+    "metric": Workload("metric", B=64, Sq=1, H=128, L=8192, seed=1005),
+}
+
+
+def _stream_seed(seed: int, b: int, which: int) -> int:
+    # distinct, reproducible generator per (workload seed, sequence, tensor)
+    return (seed * 1_000_003 + b * 4 + which) & ((1 << 62) - 1)
+
+
+def make_q(w: Workload, b: int) -> torch.Tensor:
+    g = torch.Generator().manual_seed(_stream_seed(w.seed, b, 0))
+    return (torch.randn(w.Sq, w.H, D_QK, generator=g) * w.sigma).to(torch.bfloat16)
+
+
+def make_kv_rows(w: Workload, b: int, n_rows: int) -> torch.Tensor:
+    g = torch.Generator().manual_seed(_stream_seed(w.seed, b, 1))
+    return (torch.randn(n_rows, D_QK, generator=g) * w.sigma).to(torch.bfloat16)
+
+
+def generate(w: Workload, tail_fill: float = float("nan"), lengths: Optional[torch.Tensor] = None):
+    """Materialise (q [B,Sq,H,576], kv [B,L_max,576], seqlens [B]) on the CPU."""
+    sl = w.lengths() if lengths is None else lengths.to(torch.int32)
+    q = torch.empty((w.B, w.Sq, w.H, D_QK), dtype=torch.bfloat16)
+    kv = torch.empty((w.B, w.L, D_QK), dtype=torch.bfloat16)
+    for b in range(w.B):
+        q[b] = make_q(w, b)
+        Lb = int(sl[b])
+        if Lb > 0:
+            kv[b, :Lb] = make_kv_rows(w, b, Lb)
+        if Lb < w.L:
+            kv[b, Lb:] = tail_fill
+    return q, kv, sl
+
+
+def small_variant(w: Workload, B: Optional[int] = None, L: Optional[int] = None,
+                  L_lo: Optional[int] = None, seed_offset: int = 0) -> Workload:
+    """Same head layout and value distribution at a size the oracle finishes quickly."""
+    return dataclasses.replace(w, name=w.name + "_small", B=B or w.B, L=L or w.L,
+                               L_lo=L_lo if w.L_lo is not None else None,
+                               seed=w.seed + seed_offset)
+
+
+def custom(B: int, Sq: int, H: int, L: int, L_lo: Optional[int] = None,
+           sigma: float = 1.0, seed: int = 7) -> Workload:
+    return Workload(f"custom_B{B}_Sq{Sq}_H{H}_L{L}", B=B, Sq=Sq, H=H, L=L, L_lo=L_lo,
+                    sigma=sigma, seed=seed)
+
+
+def ceil_div(a: int, b: int) -> int:
+    return -(-a // b)
+
+
+__all__ = ["Workload", "WORKLOADS", "generate", "make_q", "make_kv_rows", "small_variant",
+           "custom", "D_QK", "D_V", "D_ROPE", "ceil_div"]

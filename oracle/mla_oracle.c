@@ -1,0 +1,194 @@
+/*
+ * mla_oracle.c -- plain fp64 CPU oracle for Multi-head Latent Attention (MLA)
+ * decode.  TEST INFRASTRUCTURE ONLY: tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py are the only callers.  The CUDA
+ * library never links, loads or calls this file, and this file uses nothing
+ * from the CUDA library (no shared headers, helpers, tables or constants).
+ *
+ * What it computes.  MLA decode is the running example, ablation subject and
+ * headline benchmark of "TileLang: Bridging Programmability and Performance in
+ * Modern Neural Kernels" (papernotes.org summary, section "一个完整示例：FlashMLA
+ * 的两阶段优化" and the main-results table "主实验", row FlashMLA); the hackmd
+ * essay "TileLang 完整解析" benchmarks it in section "FlashMLA Benchmark".  The
+ * pages describe the kernel as two GEMMs around a softmax (S = Q K^T, then
+ * P V) but never write the formula, so this file writes out the textbook
+ * definition of scaled-dot-product attention over a shared latent cache:
+ *
+ *   for every sequence b, query token t < Sq, head h < H, with L = seqlens[b]:
+ *     s_j          = scale * sum_{d < d_qk} q[b,t,h,d] * kv[b,j,d]      (j < L)
+ *     m            = max_j s_j
+ *     l            = sum_j exp(s_j - m)
+ *     out[b,t,h,e] = sum_j exp(s_j - m) * kv[b,j,e] / l                (e < d_v)
+ *     lse[b,t,h]   = m + ln(l)                                   (natural log)
+ *
+ * Keys are the d_qk-wide latent rows (512 latent + 64 rope = 576 for MLA) and
+ * the values are the first d_v (= 512) columns of the very same rows.  The Sq
+ * query tokens of a sequence all see keys 0..L-1 (no mask between them).  An
+ * empty sequence (L = 0) gives out = 0 and lse = -inf.
+ *
+ * Arithmetic: every bf16 input is widened exactly to double; sums run in
+ * index order in double; exp/log are the C library's double routines.  Two
+ * passes (max, then sum): no base-2 trick, no online rescaling, no splitting,
+ * no blocking.  Parallelism: OpenMP over independent (b, t, h) rows only.
+ *
+ * Parity pins (tests/test_oracle.py, CPU only): closed forms (single key,
+ * identical keys, q = 0, two keys), invariants (permutation of keys, a shared
+ * additive score shift, head and token independence), brute force in 50-digit
+ * decimal arithmetic on tiny shapes, and torch's fp64 scaled_dot_product_
+ * attention as an independent library routine.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Exact widening of a bfloat16 bit pattern: bf16 is the top half of an IEEE
+ * binary32, so shifting the bits up gives the float, and float -> double is
+ * exact. */
+static double bf16_bits_to_double(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* One output row (b, t, h): the definition above, written out. `scores` is a
+ * caller-owned scratch array of at least L doubles. */
+static void attend_one_row(const uint16_t *q_row, const uint16_t *kv_seq,
+                           int64_t L, int64_t d_qk, int64_t d_v, double scale,
+                           double *scores, double *out_row, double *lse_out)
+{
+    if (L <= 0) {
+        for (int64_t e = 0; e < d_v; ++e) out_row[e] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    /* s_j = scale * <q, k_j> over all d_qk columns (latent + rope). */
+    for (int64_t j = 0; j < L; ++j) {
+        const uint16_t *k_row = kv_seq + j * d_qk;
+        double dot = 0.0;
+        for (int64_t d = 0; d < d_qk; ++d)
+            dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(k_row[d]);
+        scores[j] = scale * dot;
+    }
+    /* m = max_j s_j */
+    double m = scores[0];
+    for (int64_t j = 1; j < L; ++j)
+        if (scores[j] > m) m = scores[j];
+    /* w_j = exp(s_j - m), l = sum_j w_j */
+    double l = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+        scores[j] = exp(scores[j] - m);
+        l += scores[j];
+    }
+    /* out_e = sum_j w_j * v_j[e] / l, with v_j = first d_v columns of row j */
+    for (int64_t e = 0; e < d_v; ++e) out_row[e] = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+        const uint16_t *v_row = kv_seq + j * d_qk;
+        const double w = scores[j];
+        for (int64_t e = 0; e < d_v; ++e)
+            out_row[e] += w * bf16_bits_to_double(v_row[e]);
+    }
+    for (int64_t e = 0; e < d_v; ++e) out_row[e] /= l;
+    *lse_out = m + log(l);
+}
+
+/*
+ * Full oracle.
+ *   q       : bf16 bits, [B, Sq, H, d_qk] contiguous
+ *   kv      : bf16 bits, [B, L_max, d_qk] contiguous (values = first d_v cols)
+ *   seqlens : int32 [B], 0 <= seqlens[b] <= L_max
+ *   out     : double [B, Sq, H, d_v];  lse : double [B, Sq, H]
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
+ */
+int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                      int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                      int64_t d_qk, int64_t d_v, double scale,
+                      double *out, double *lse, int num_threads)
+{
+    if (!q || !kv || !seqlens || !out || !lse) return -1;
+    if (B < 0 || Sq < 1 || H < 1 || L_max < 0 || d_qk < 1 || d_v < 1 || d_v > d_qk) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > L_max) return -1;
+    const int64_t rows = B * Sq * H;
+    int failed = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(L_max > 0 ? L_max : 1));
+        if (!scores) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < rows; ++r) {
+                const int64_t b = r / (Sq * H);
+                attend_one_row(q + r * d_qk, kv + b * L_max * d_qk, seqlens[b],
+                               d_qk, d_v, scale, scores, out + r * d_v, lse + r);
+            }
+            free(scores);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Sampled oracle: the same definition for a caller-chosen list of flattened
+ * row indices r = (b * Sq + t) * H + h, so that full-size workloads can be
+ * checked row by row.  out is [n_rows, d_v], lse is [n_rows].
+ */
+int oracle_mla_decode_rows(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                           int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                           int64_t d_qk, int64_t d_v, double scale,
+                           const int64_t *row_ids, int64_t n_rows,
+                           double *out, double *lse, int num_threads)
+{
+    if (!q || !kv || !seqlens || !row_ids || !out || !lse) return -1;
+    if (B < 0 || Sq < 1 || H < 1 || L_max < 0 || d_qk < 1 || d_v < 1 || d_v > d_qk) return -1;
+    for (int64_t i = 0; i < n_rows; ++i)
+        if (row_ids[i] < 0 || row_ids[i] >= B * Sq * H) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > L_max) return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(L_max > 0 ? L_max : 1));
+        if (!scores) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t i = 0; i < n_rows; ++i) {
+                const int64_t r = row_ids[i];
+                const int64_t b = r / (Sq * H);
+                attend_one_row(q + r * d_qk, kv + b * L_max * d_qk, seqlens[b],
+                               d_qk, d_v, scale, scores, out + i * d_v, lse + i);
+            }
+            free(scores);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/* Number of OpenMP threads a parallel region of this library would use. */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,235 @@
+"""Checks that pin the fp64 oracle to facts other than itself.
+
+Each ``pin_*`` takes an implementation ``impl(q, kv, seqlens, scale, d_v) ->
+(out, lse)`` (numpy float64 results) and raises AssertionError when the
+implementation disagrees with a closed form, an invariant fixed by the
+definition, a high-precision brute force, or an independent library routine.
+tests/test_oracle.py runs them on the oracle, and also on deliberately broken
+variants to show that each plausible mistake trips at least one pin.
+"""
+from __future__ import annotations
+
+import math
+from decimal import Decimal, getcontext
+
+import numpy as np
+import torch
+
+SCALE = float(torch.tensor(576 ** -0.5, dtype=torch.float32).item())
+
+
+def _rand_bf16(shape, gen, sigma=1.0):
+    return (torch.randn(*shape, generator=gen) * sigma).to(torch.bfloat16)
+
+
+def _f64(x):
+    return x.to(torch.float64).numpy()
+
+
+def pin_single_key(impl):
+    """L = 1: the only weight is 1, so out is that key's value row and lse is
+    its scaled score."""
+    g = torch.Generator().manual_seed(11)
+    q = _rand_bf16((2, 1, 4, 576), g)
+    kv = _rand_bf16((2, 3, 576), g)
+    sl = np.array([1, 1], dtype=np.int32)
+    out, lse = impl(q, kv, sl, SCALE, 512)
+    for b in range(2):
+        for h in range(4):
+            np.testing.assert_array_equal(out[b, 0, h], _f64(kv[b, 0, :512]))
+            s0 = SCALE * float(torch.dot(q[b, 0, h].double(), kv[b, 0].double()))
+            assert abs(lse[b, 0, h] - s0) <= 1e-12 * max(1.0, abs(s0))
+
+
+def pin_identical_keys(impl):
+    """L identical rows: uniform weights, out = that row's value, lse = s + ln L."""
+    g = torch.Generator().manual_seed(12)
+    q = _rand_bf16((1, 1, 3, 576), g)
+    row = _rand_bf16((576,), g)
+    L = 37
+    kv = row.expand(1, L, 576).contiguous()
+    out, lse = impl(q, kv, np.array([L], np.int32), SCALE, 512)
+    for h in range(3):
+        np.testing.assert_allclose(out[0, 0, h], _f64(row[:512]), rtol=0, atol=1e-14)
+        s = SCALE * float(torch.dot(q[0, 0, h].double(), row.double()))
+        assert abs(lse[0, 0, h] - (s + math.log(L))) <= 1e-12
+
+
+def pin_zero_query(impl):
+    """q = 0: all scores are 0, weights uniform: out = mean of value rows,
+    lse = ln L."""
+    g = torch.Generator().manual_seed(13)
+    q = torch.zeros((2, 1, 2, 576), dtype=torch.bfloat16)
+    kv = _rand_bf16((2, 50, 576), g)
+    sl = np.array([50, 17], np.int32)
+    out, lse = impl(q, kv, sl, SCALE, 512)
+    for b, L in enumerate(sl):
+        mean = kv[b, :L, :512].double().mean(dim=0).numpy()
+        for h in range(2):
+            np.testing.assert_allclose(out[b, 0, h], mean, rtol=0, atol=1e-13)
+            assert abs(lse[b, 0, h] - math.log(L)) <= 1e-13
+
+
+def pin_two_keys(impl):
+    """Closed form: q = a e_0, k_0 = e_0, k_1 = e_1 (q . k_1 = 0): weights
+    sigma(a*scale) and 1 - sigma(a*scale); lse = ln(exp(a*scale) + 1)."""
+    a = 6.5  # exactly representable in bf16
+    q = torch.zeros((1, 1, 1, 576), dtype=torch.bfloat16)
+    q[0, 0, 0, 0] = a
+    g = torch.Generator().manual_seed(14)
+    kv = _rand_bf16((1, 2, 576), g)
+    kv[0, 0, :] = 0
+    kv[0, 1, :] = 0
+    kv[0, 0, 0] = 1.0
+    kv[0, 1, 1] = 1.0
+    v0 = torch.zeros(512, dtype=torch.float64)
+    v0[0] = 1.0
+    v1 = torch.zeros(512, dtype=torch.float64)
+    v1[1] = 1.0
+    z = a * SCALE
+    w0 = 1.0 / (1.0 + math.exp(-z))
+    out, lse = impl(q, kv, np.array([2], np.int32), SCALE, 512)
+    np.testing.assert_allclose(out[0, 0, 0], (w0 * v0 + (1 - w0) * v1).numpy(), rtol=0, atol=1e-15)
+    assert abs(lse[0, 0, 0] - math.log(math.exp(z) + 1.0)) <= 1e-14
+
+
+def pin_rope_shift(impl):
+    """A shared additive score term: setting the last rope column of q to 1 and
+    of every key to 2 adds 2*scale to every score, which leaves out unchanged
+    and shifts lse by exactly 2*scale (and proves the rope columns count)."""
+    g = torch.Generator().manual_seed(15)
+    q = _rand_bf16((1, 1, 4, 576), g)
+    kv = _rand_bf16((1, 29, 576), g)
+    q[..., 575] = 0
+    kv[..., 575] = 0
+    out0, lse0 = impl(q, kv, np.array([29], np.int32), SCALE, 512)
+    q[..., 575] = 1.0
+    kv[..., 575] = 2.0
+    out1, lse1 = impl(q, kv, np.array([29], np.int32), SCALE, 512)
+    np.testing.assert_allclose(out1, out0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse1 - lse0, 2.0 * SCALE, rtol=0, atol=1e-12)
+
+
+def pin_value_columns(impl):
+    """Values are the first 512 columns: with every key equal except for
+    columns >= 512, the output must be identical (those columns feed scores
+    only), and changing column 0 of one key must move out[..., 0]."""
+    g = torch.Generator().manual_seed(16)
+    q = torch.zeros((1, 1, 1, 576), dtype=torch.bfloat16)
+    kv = _rand_bf16((1, 5, 576), g)
+    out, _ = impl(q, kv, np.array([5], np.int32), SCALE, 512)
+    mean = kv[0, :5, :512].double().mean(dim=0).numpy()
+    np.testing.assert_allclose(out[0, 0, 0], mean, rtol=0, atol=1e-13)
+    kv2 = kv.clone()
+    kv2[0, :, 512:] = 0  # rope columns never contribute to values
+    out2, _ = impl(q, kv2, np.array([5], np.int32), SCALE, 512)
+    np.testing.assert_allclose(out2, out, rtol=0, atol=1e-15)
+
+
+def pin_permutation(impl):
+    """Reordering the keys (with their values) leaves out and lse unchanged."""
+    g = torch.Generator().manual_seed(17)
+    q = _rand_bf16((1, 2, 3, 576), g)
+    kv = _rand_bf16((1, 41, 576), g)
+    perm = torch.randperm(41, generator=g)
+    out0, lse0 = impl(q, kv, np.array([41], np.int32), SCALE, 512)
+    out1, lse1 = impl(q, kv[:, perm].contiguous(), np.array([41], np.int32), SCALE, 512)
+    np.testing.assert_allclose(out1, out0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse1, lse0, rtol=0, atol=1e-13)
+
+
+def pin_independence(impl):
+    """Rows do not interact: each (token, head) equals a run on that row alone,
+    and each sequence sees only its own cache and length."""
+    g = torch.Generator().manual_seed(18)
+    q = _rand_bf16((2, 2, 3, 576), g)
+    kv = _rand_bf16((2, 23, 576), g)
+    sl = np.array([23, 9], np.int32)
+    out, lse = impl(q, kv, sl, SCALE, 512)
+    for b in range(2):
+        for t in range(2):
+            for h in range(3):
+                o1, l1 = impl(q[b:b + 1, t:t + 1, h:h + 1].contiguous(), kv[b:b + 1].contiguous(),
+                              sl[b:b + 1], SCALE, 512)
+                np.testing.assert_allclose(o1[0, 0, 0], out[b, t, h], rtol=0, atol=1e-14)
+                assert abs(l1[0, 0, 0] - lse[b, t, h]) <= 1e-14
+
+
+def pin_tail_ignored(impl):
+    """Rows at or past a sequence's length are never read (NaN there changes
+    nothing), and an empty sequence gives out = 0, lse = -inf."""
+    g = torch.Generator().manual_seed(19)
+    q = _rand_bf16((3, 1, 2, 576), g)
+    kv = _rand_bf16((3, 16, 576), g)
+    sl = np.array([16, 5, 0], np.int32)
+    out0, lse0 = impl(q, kv, sl, SCALE, 512)
+    kv_nan = kv.clone()
+    kv_nan[1, 5:] = float("nan")
+    kv_nan[2, :] = float("nan")
+    out1, lse1 = impl(q, kv_nan, sl, SCALE, 512)
+    np.testing.assert_array_equal(out1, out0)
+    np.testing.assert_array_equal(lse1, lse0)
+    assert np.all(out1[2] == 0.0) and np.all(np.isneginf(lse1[2]))
+
+
+def _decimal_reference(q, kv, sl, scale, d_v, digits=50):
+    getcontext().prec = digits
+    qd = q.to(torch.float64).numpy()
+    kd = kv.to(torch.float64).numpy()
+    B, Sq, H, d = qd.shape
+    out = np.zeros((B, Sq, H, d_v))
+    lse = np.zeros((B, Sq, H))
+    sc = Decimal(scale)
+    for b in range(B):
+        L = int(sl[b])
+        for t in range(Sq):
+            for h in range(H):
+                s = [sc * sum(Decimal(float(qd[b, t, h, i])) * Decimal(float(kd[b, j, i])) for i in range(d))
+                     for j in range(L)]
+                m = max(s)
+                w = [(x - m).exp() for x in s]
+                l = sum(w)
+                for e in range(d_v):
+                    out[b, t, h, e] = float(sum(w[j] * Decimal(float(kd[b, j, e])) for j in range(L)) / l)
+                lse[b, t, h] = float(m + l.ln())
+    return out, lse
+
+
+def pin_brute_force_decimal(impl):
+    """50-digit decimal brute force on tiny shapes (d_qk = 6, d_v = 4), with
+    generic dimensions, large score spread and ragged lengths."""
+    g = torch.Generator().manual_seed(20)
+    q = _rand_bf16((2, 2, 2, 6), g, sigma=3.0)
+    kv = _rand_bf16((2, 5, 6), g, sigma=3.0)
+    sl = np.array([5, 3], np.int32)
+    scale = 0.37
+    out, lse = impl(q, kv, sl, scale, 4)
+    ro, rl = _decimal_reference(q, kv, sl, scale, 4)
+    np.testing.assert_allclose(out, ro, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-13)
+
+
+def pin_sdpa_library(impl):
+    """torch's fp64 scaled_dot_product_attention (math path) with k = kv rows
+    and v = their first 512 columns, and torch.logsumexp of the fp64 scores for
+    lse, at the real 576/512 dimensions with ragged lengths and two tokens."""
+    g = torch.Generator().manual_seed(21)
+    q = _rand_bf16((2, 2, 4, 576), g)
+    kv = _rand_bf16((2, 67, 576), g)
+    sl = np.array([67, 30], np.int32)
+    out, lse = impl(q, kv, sl, SCALE, 512)
+    for b in range(2):
+        L = int(sl[b])
+        qq = q[b].double().reshape(1, -1, 576)           # [1, Sq*H, 576]
+        kk = kv[b, :L].double().reshape(1, L, 576)
+        vv = kv[b, :L, :512].double().reshape(1, L, 512)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=SCALE)
+        np.testing.assert_allclose(out[b].reshape(-1, 512), ref[0].numpy(), rtol=0, atol=1e-12)
+        scores = (qq[0] @ kk[0].T) * SCALE
+        np.testing.assert_allclose(lse[b].reshape(-1), torch.logsumexp(scores, dim=-1).numpy(),
+                                   rtol=0, atol=1e-12)
+
+
+ALL_PINS = [pin_single_key, pin_identical_keys, pin_zero_query, pin_two_keys, pin_rope_shift,
+            pin_value_columns, pin_permutation, pin_independence, pin_tail_ignored,
+            pin_brute_force_decimal, pin_sdpa_library]

@@ -1,0 +1,130 @@
+"""The fp64 oracle against its pins (CPU only), and the pins' own sensitivity:
+each plausible mistake, planted in a CPU stand-in of the oracle, must trip at
+least one pin."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import oracle_pins as pins
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def oracle_impl(q, kv, sl, scale, d_v):
+    return oracle.mla_decode(q, kv, sl, scale, d_v=d_v)
+
+
+@pytest.mark.parametrize("pin", pins.ALL_PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(pin):
+    pin(oracle_impl)
+
+
+def test_rows_entry_matches_full():
+    g = torch.Generator().manual_seed(3)
+    q = (torch.randn(3, 2, 5, 576, generator=g)).to(torch.bfloat16)
+    kv = (torch.randn(3, 40, 576, generator=g)).to(torch.bfloat16)
+    sl = np.array([40, 1, 0], np.int32)
+    out, lse = oracle.mla_decode(q, kv, sl, pins.SCALE)
+    rows = np.array([0, 7, 12, 13, 29, 10], np.int64)
+    o2, l2 = oracle.mla_decode_rows(q, kv, sl, pins.SCALE, rows)
+    np.testing.assert_array_equal(o2, out.reshape(-1, 512)[rows])
+    np.testing.assert_array_equal(l2, lse.reshape(-1)[rows])
+
+
+def test_rejects_bad_lengths():
+    q = torch.zeros(1, 1, 1, 576, dtype=torch.bfloat16)
+    kv = torch.zeros(1, 4, 576, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        oracle.mla_decode(q, kv, np.array([5], np.int32), pins.SCALE)
+    with pytest.raises(ValueError):
+        oracle.mla_decode(q, kv, np.array([-1], np.int32), pins.SCALE)
+
+
+def test_golden_fixture_reproduces():
+    """tests/golden/tiny_oracle.json was written by tests/golden/make_golden.py,
+    which calls only oracle/; the oracle must keep reproducing it."""
+    from mla_decode_attention_11_b200 import workloads as W
+    with open(os.path.join(GOLDEN, "tiny_oracle.json")) as f:
+        gold = json.load(f)
+    w = W.WORKLOADS[gold["workload"]]
+    q, kv, sl = W.generate(w)
+    out, lse = oracle.mla_decode(q, kv, sl, w.scale)
+    np.testing.assert_allclose(lse.reshape(-1), np.array(gold["lse"]), rtol=0, atol=1e-12)
+    flat = out.reshape(-1)
+    idx = np.array(gold["out_index"], dtype=np.int64)
+    np.testing.assert_allclose(flat[idx], np.array(gold["out_value"]), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- mutants
+# CPU stand-ins of the oracle with one planted mistake each.  They are never
+# used as references; they exist only to show the pins would catch the mistake.
+
+def _np_attention(q, kv, sl, scale, d_v, *, qk_cols=None, v_cols=None, lse_base=math.e,
+                  scale_used=True, sign=1.0, len_delta=0, add_max_to_lse=True,
+                  normalise=True, head_mixup=False):
+    qd = q.to(torch.float64).numpy()
+    kd = kv.to(torch.float64).numpy()
+    B, Sq, H, d = qd.shape
+    out = np.zeros((B, Sq, H, d_v))
+    lse = np.zeros((B, Sq, H))
+    qc = slice(0, d) if qk_cols is None else qk_cols
+    vc = slice(0, d_v) if v_cols is None else slice(d - d_v, d)  # "last d_v columns"
+    for b in range(B):
+        L = int(sl[b]) + len_delta
+        L = max(0, min(L, kd.shape[1]))
+        for t in range(Sq):
+            for h in range(H):
+                if L == 0:
+                    lse[b, t, h] = -np.inf
+                    continue
+                qrow = qd[b, t, 0 if head_mixup else h]
+                s = sign * (kd[b, :L, qc] @ qrow[qc]) * (scale if scale_used else 1.0)
+                m = s.max()
+                w = np.exp(s - m)
+                l = w.sum()
+                o = w @ kd[b, :L, vc]
+                out[b, t, h] = o / l if normalise else o
+                lse[b, t, h] = ((m if add_max_to_lse else 0.0) + np.log(l)) / math.log(lse_base)
+    return out, lse
+
+
+MUTANTS = {
+    "correct": {},
+    "drop_rope_columns": dict(qk_cols=slice(0, 512)),
+    "values_from_last_columns": dict(v_cols="last"),
+    "lse_in_base_2": dict(lse_base=2.0),
+    "scale_ignored": dict(scale_used=False),
+    "score_sign_flipped": dict(sign=-1.0),
+    "one_key_short": dict(len_delta=-1),
+    "one_key_past_end": dict(len_delta=+1),
+    "max_missing_from_lse": dict(add_max_to_lse=False),
+    "output_not_normalised": dict(normalise=False),
+    "heads_mixed_up": dict(head_mixup=True),
+}
+
+
+def _run_pins(kwargs):
+    def impl(q, kv, sl, scale, d_v):
+        return _np_attention(q, kv, sl, scale, d_v, **kwargs)
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistakes(name):
+    failed = _run_pins(MUTANTS[name])
+    if name == "correct":
+        assert failed == [], f"a correct stand-in must pass every pin, failed: {failed}"
+    else:
+        assert failed, f"planted mistake '{name}' passed every pin"
