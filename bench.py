@@ -1,0 +1,352 @@
+#!/usr/bin/env python
+"""MLA decode benchmark on B200: TFLOP/s, HBM GB/s and the roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload metric] [--impl ours|reference]
+
+A step is one full MLA decode (main kernel + split-KV combine) of the
+workload with inputs already resident in HBM.  The default workload is the
+headline line: B=64 sequences, Sq=1, H=128 heads, every L=8192, d_qk=576,
+d_v=512, bf16 N(0,1) seeded synthetic data; its kv (604 MB) is larger than
+the 126 MB L2, so no flush is needed between steps.  Prints ONE JSON line on
+rank 0.  Under torchrun (N > 1) every rank runs an independent replica (the
+path has no cross-GPU exchange); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+this path) on a bounded sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from mla_decode_attention_11_b200 import workloads as W  # noqa: E402
+
+METRIC = "MLA decode TFLOP/s + HBM GB/s at B=64,H=128,L=8192; fraction of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    from mla_decode_attention_11_b200 import build as B
+    h = hashlib.sha256()
+    for s in B.sources():
+        with open(s, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per main-kernel launch from a committed ncu summary, used only
+    if it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None, None
+    with open(path) as f:
+        d = json.load(f)
+    ent = d.get(workload)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None, None
+    return float(ent["dram_bytes_per_launch"]), ent.get("note")
+
+
+def workload_desc(w: W.Workload) -> str:
+    L = f"U[{w.L_lo},{w.L}]" if w.L_lo is not None else f"{w.L} (all)"
+    return (f"{w.name}: B={w.B} Sq={w.Sq} H={w.H} L={L}, d_qk=576 (512 latent + 64 rope), d_v=512, "
+            f"bf16 N(0,{w.sigma:g}) seed {w.seed}, scale 576^-0.5")
+
+
+class ClockSampler:
+    """Polls SM clock / throttle reasons through NVML during the timed region."""
+
+    REASONS = {0x0000000000000004: "sw_power_cap", 0x0000000000000008: "hw_slowdown",
+               0x0000000000000020: "sw_thermal_slowdown", 0x0000000000000040: "hw_thermal_slowdown",
+               0x0000000000000080: "hw_power_brake_slowdown", 0x0000000000000001: "gpu_idle",
+               0x0000000000000002: "applications_clocks_setting", 0x0000000000000100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            u = str(uuid)
+            if not u.startswith("GPU-"):
+                u = "GPU-" + u
+            try:
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(u)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        if self._thr:
+            self._stop.set()
+            self._thr.join()
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def cpu_oracle_sample(w: W.Workload, q, kv, sl, seqs):
+    """Time the oracle, as it stands, on whole sequences `seqs` (all heads)."""
+    import numpy as np
+    import oracle
+    R = w.Sq * w.H
+    rows = np.concatenate([np.arange(b * R, (b + 1) * R) for b in seqs]).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.mla_decode_rows(q, kv, sl, w.scale, rows)
+    dt = time.perf_counter() - t0
+    flops = sum(int(sl[b]) for b in seqs) * R * 2 * (W.D_QK + W.D_V)
+    return flops, dt, oracle.max_threads()
+
+
+def run_reference(args, w: W.Workload):
+    """--impl reference: the fp64 CPU oracle on a bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    q, kv, sl = W.generate(w, tail_fill=0.0)
+    seqs_per_step = 1
+    for i in range(args.warmup):
+        cpu_oracle_sample(w, q, kv, sl, [i % w.B])
+    tot_flops, tot_t, cores = 0, 0.0, 1
+    for i in range(args.steps):
+        f, dt, cores = cpu_oracle_sample(w, q, kv, sl, [(args.warmup + i) % w.B])
+        tot_flops += f
+        tot_t += dt
+    value = tot_flops / tot_t / 1e12
+    sample = (f"{seqs_per_step} whole sequence per step ({w.Sq * w.H} query rows x L={w.L}) of the "
+              f"{w.B}-sequence workload, {args.steps} steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "parallelism": "host cores (OpenMP)", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w: W.Workload):
+    from mla_decode_attention_11_b200 import binding as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    q, kv, sl = W.generate(w, tail_fill=0.0)
+    qd, kvd, sld = q.to(dev), kv.to(dev), sl.to(dev)
+    plan = M.mla_decode_plan(w.B, w.Sq, w.H, w.L, device=local)
+    ws = M.alloc_workspace(plan, device=dev)
+    M.mla_decode_workspace_init(plan, ws)
+    out = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        M.mla_decode_run(plan, qd, kvd, sld, w.scale, out, lse, ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    M.mla_decode_check(plan, ws, stream=stream)
+
+    # ---- timed region: K full steps
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if dist:
+        dist.barrier()
+    t_ms = e0.elapsed_time(e1) / args.steps
+    M.mla_decode_check(plan, ws, stream=stream)
+    if dist:
+        t = torch.tensor([t_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_ms = float(t.item())
+
+    # ---- per-kernel breakdown (same work: phase 1 = main kernel, phase 2 = combine)
+    main_ms, comb_ms = [], []
+    for _ in range(max(3, min(args.steps, 50))):
+        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        a.record(stream)
+        M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, 1, stream=stream)
+        b.record(stream)
+        M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, 2, stream=stream)
+        c.record(stream)
+        torch.cuda.synchronize(dev)
+        main_ms.append(a.elapsed_time(b))
+        comb_ms.append(b.elapsed_time(c))
+    main_avg = statistics.mean(main_ms)
+    comb_avg = statistics.mean(comb_ms)
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, 5))
+    qh, kvh, slh = q.pin_memory(), kv.pin_memory(), sl.pin_memory()
+    outh = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16).pin_memory()
+    lseh = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32).pin_memory()
+    bufs = {}
+    M.mla_decode_host(qh, kvh, slh, w.scale, plan, ws, dev_bufs=bufs, out_host=outh, lse_host=lseh)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(e2e_steps):
+        M.mla_decode_host(qh, kvh, slh, w.scale, plan, ws, dev_bufs=bufs, out_host=outh, lse_host=lseh)
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = q.numel() * 2 + kv.numel() * 2 + sl.numel() * 4
+    d2h = outh.numel() * 2 + lseh.numel() * 4
+    M.mla_decode_check(plan, ws, stream=stream)
+
+    flops = w.algorithmic_flops(sl)
+    nbytes = w.algorithmic_bytes(sl)
+    peaks, peak_src = load_peaks()
+    value = world * flops / (t_ms * 1e-3) / 1e12
+    hbm_gbs = world * nbytes / (t_ms * 1e-3) / 1e9
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    ai = flops / nbytes
+    bound = "hbm" if ai < ridge else "tensor"
+    if bound == "hbm":
+        achieved = nbytes / (main_avg * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    else:
+        achieved = flops / (main_avg * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    roof_time_ms = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e3
+    traffic, traffic_note = load_traffic(w.name)
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_seq = 8 if w.H * w.Sq * w.L >= 128 * 8192 else max(1, min(w.B, 32))
+        seqs = list(range(0, w.B, max(1, w.B // n_seq)))[:n_seq]
+        f_cpu, dt_cpu, cores = cpu_oracle_sample(w, q, kv, sl, seqs)
+        cpu_base = {"value": f_cpu / dt_cpu / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                    "sample": f"{len(seqs)} of {w.B} sequences, all {w.Sq * w.H} query rows, "
+                              f"{dt_cpu:.1f} s of fp64 CPU work"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.L,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "kernel": {1: "transposed", 2: "pair"}.get(plan.kernel, str(plan.kernel)),
+                       "group_rows": plan.group_rows, "partitions": plan.num_partitions,
+                       "l2": "inputs larger than L2 (kv %.0f MB > 126 MB), no flush" % (kv.numel() * 2 / 1e6)},
+            "hbm_gbs": hbm_gbs,
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else peak_src,
+                         "kernel": "mla_decode_transposed_kernel" if plan.kernel == 1 else "mla_decode_pair_kernel",
+                         "kernel_ms": main_avg, "combine_ms": comb_avg,
+                         "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                         "tensor_tflops": flops / (main_avg * 1e-3) / 1e12,
+                         "tensor_frac": flops / (main_avg * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                         "step_roofline_frac": roof_time_ms / t_ms, "traffic_note": traffic_note},
+            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu_base,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="metric", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

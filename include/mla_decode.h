@@ -1,0 +1,186 @@
+/*
+ * mla_decode.h -- C ABI of the B200 (sm_100a) Multi-head Latent Attention
+ * decode library (libmla_decode.so).
+ *
+ * The operation.  MLA decode is the running example, ablation subject and
+ * headline kernel of "TileLang: Bridging Programmability and Performance in
+ * Modern Neural Kernels" (papernotes.org summary: section "一个完整示例：FlashMLA
+ * 的两阶段优化" describes it as a first GEMM S = Q K^T with Q and the KV tile in
+ * shared memory, a softmax over S, and a second GEMM of the cast scores with
+ * V; the main-results table "主实验", row FlashMLA, and the hackmd essay
+ * "TileLang 完整解析", section "FlashMLA Benchmark", time it).  The pages leave
+ * the formula to the reader; this library computes the textbook definition:
+ * for every sequence b, query token t < Sq and head h < H, with L = seqlens[b],
+ *
+ *     s_j          = softmax_scale * sum_{d<576} q[b,t,h,d] * kv[b,j,d]    (j < L)
+ *     out[b,t,h,e] = sum_j exp(s_j - max s) kv[b,j,e] / sum_j exp(s_j - max s)  (e < 512)
+ *     lse[b,t,h]   = ln sum_j exp(s_j)                          (natural log)
+ *
+ * i.e. many query heads attend over ONE shared compressed latent cache whose
+ * rows are 576 wide (512 latent + 64 rope); the values are the first 512
+ * columns of the same rows.  The Sq query tokens of a sequence all see keys
+ * 0..L-1 (no mask between them).  L = 0 gives out = 0 and lse = -inf.
+ *
+ * Numerics: bf16 inputs, fp32 accumulation in the tensor cores, fp32 online
+ * softmax in base 2 (as in the online-softmax fragment of "DeepSeekV4-
+ * TileLang", qingkeai.online, section "TileLang 的设计精髓"), bf16 output.
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory.  The library never allocates device memory;
+ *     it keeps no global state besides a per-process cache of the CUDA driver
+ *     entry point it uses to encode TMA descriptors.
+ *   - Pointers named "device" must be device pointers of the plan's device;
+ *     "host" pointers are ordinary host memory.
+ *   - Work is enqueued on `stream` and runs asynchronously; a return of MLA_OK
+ *     means the arguments were valid and the launches were accepted.  Faults
+ *     detected on the device (timeouts, lengths out of range) are recorded in
+ *     the workspace and reported by mla_decode_check().
+ *   - No entry point throws, aborts or prints.
+ */
+#ifndef MLA_DECODE_H_
+#define MLA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mla_status {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,   /* a null pointer, a size out of range, an inconsistent plan */
+    MLA_ERR_ALIGNMENT = 2,     /* a pointer not 16-byte aligned (TMA needs 16-byte aligned bases) */
+    MLA_ERR_UNSUPPORTED = 3,   /* a shape this build has no kernel for (see mla_decode_plan) */
+    MLA_ERR_CUDA = 4,          /* a CUDA runtime / driver call failed (launch, attribute, ...) */
+    MLA_ERR_TIMEOUT = 5,       /* device: a bounded pipeline wait ran out; results are invalid */
+    MLA_ERR_WORKSPACE = 6,     /* workspace pointer null or smaller than the plan requires */
+    MLA_ERR_SEQLEN = 7         /* device: some seqlens[b] was < 0 or > L_max (clamped to [0, L_max]) */
+} mla_status;
+
+/* Kernel variants a plan can select. */
+enum {
+    MLA_KERNEL_TRANSPOSED = 1, /* S^T = K Q^T per CTA, kv rows on the 128 TMEM lanes (any H*Sq) */
+    MLA_KERNEL_PAIR = 2        /* CTA pair, 64 query rows per CTA, cta_group::2 MMAs (H*Sq % 128 == 0) */
+};
+
+/*
+ * Launch plan.  Filled by mla_decode_plan(); treat as read-only.  Plain data:
+ * it may be copied, kept for any number of runs and freed by the caller.
+ */
+typedef struct mla_plan {
+    int32_t B, Sq, H, L_max;   /* problem shape the plan was made for */
+    int32_t device;            /* CUDA device ordinal */
+    int32_t num_sms;           /* multiprocessors on that device */
+    int32_t kernel;            /* MLA_KERNEL_* */
+    int32_t group_rows;        /* query rows (token, head pairs) handled per CTA */
+    int32_t num_groups;        /* CTAs (or CTA pairs) that share one KV partition */
+    int32_t num_partitions;    /* KV partitions: the flattened KV tiles of all sequences are cut into
+                                  this many balanced contiguous ranges */
+    int32_t tile_kv;           /* kv rows per pipeline tile */
+    int32_t cta_threads;       /* threads per CTA of the main kernel */
+    uint64_t smem_bytes;       /* dynamic shared memory per CTA of the main kernel */
+    uint64_t workspace_bytes;  /* bytes the caller must provide to mla_decode_run */
+    uint64_t reserved[6];
+} mla_plan;
+
+/*
+ * mla_decode_plan -- validate a shape and choose kernel, grid and workspace.
+ *
+ *   B          number of sequences, 1 <= B <= 65535
+ *   Sq         query tokens per sequence, 1 <= Sq <= 16
+ *   H          query heads, one of 16, 32, 64, 128
+ *   L_max      rows allocated per sequence in kv, 1 <= L_max <= 2^24
+ *   device     CUDA device ordinal (must be an sm_100 device at run time)
+ *   num_partitions_override
+ *              0 = automatic (balanced over the device's SMs); > 0 forces that
+ *              many KV partitions (tests use it to force 1 = no split, or
+ *              many splits); it is clamped to [1, 4096]
+ *   plan       (host, out) filled on success
+ *   workspace_bytes
+ *              (host, out, may be NULL) size of the device workspace to pass
+ *              to mla_decode_run; the workspace is caller-owned, must be
+ *              256-byte aligned, and must be zeroed once (mla_decode_workspace_init)
+ *              before its first use
+ *
+ * Returns MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED or MLA_ERR_CUDA
+ * (device query failed).  Does not launch anything.
+ */
+mla_status mla_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                           int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
+
+/*
+ * mla_decode_workspace_init -- zero the workspace's status words on `stream`
+ * (asynchronous cudaMemsetAsync of the header).  Call once per workspace before
+ * the first run; mla_decode_check() re-zeroes them after reading.
+ */
+mla_status mla_decode_workspace_init(const mla_plan* plan, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/*
+ * mla_decode_run -- enqueue one MLA decode on `stream` (a cudaStream_t; NULL =
+ * the legacy default stream).
+ *
+ *   q         device, bf16 [B, Sq, H, 576], contiguous row-major, 16-byte aligned
+ *   kv        device, bf16 [B, L_max, 576], contiguous; values are kv[..., :512]
+ *   seqlens   device, int32 [B], 0 <= seqlens[b] <= L_max (rows >= seqlens[b]
+ *             are never read; out-of-range values are clamped and flagged)
+ *   softmax_scale  multiplies q.k (576^-0.5 for MLA)
+ *   out       device, bf16 [B, Sq, H, 512], contiguous, 16-byte aligned (written)
+ *   lse       device, fp32 [B, Sq, H] (written; natural-log log-sum-exp of the
+ *             scaled scores, -inf for an empty sequence)
+ *   workspace device, workspace_bytes >= plan->workspace_bytes, 256-byte aligned;
+ *             holds split-KV partial outputs and the status words.  A workspace
+ *             must not be used by two runs that may execute concurrently.
+ *
+ * Launches the main kernel and the split-KV combine kernel; no host sync, no
+ * allocation, so the call can be captured in a CUDA graph.
+ * Returns MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_ALIGNMENT, MLA_ERR_WORKSPACE,
+ * MLA_ERR_UNSUPPORTED (device is not sm_100) or MLA_ERR_CUDA.
+ */
+mla_status mla_decode_run(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                          float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/*
+ * mla_decode_run_phase -- the two launches of mla_decode_run, one at a time:
+ * phase 1 = the main kernel (partials and finished sequences), phase 2 = the
+ * split-KV combine kernel (merges partials, writes empty sequences).  Issuing
+ * phase 1 then phase 2 on one stream is exactly mla_decode_run; separate calls
+ * let a caller place events or other work between them.  Same arguments and
+ * return codes as mla_decode_run, plus MLA_ERR_INVALID_ARG for another phase.
+ */
+mla_status mla_decode_run_phase(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                                float softmax_scale, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream, int32_t phase);
+
+/*
+ * mla_decode_check -- synchronize `stream`, read and clear the workspace's
+ * device status words.  Returns MLA_OK if no run since the last check
+ * recorded a fault, else MLA_ERR_TIMEOUT / MLA_ERR_SEQLEN (the first recorded),
+ * or MLA_ERR_CUDA if the synchronization itself failed.
+ */
+mla_status mla_decode_check(const mla_plan* plan, void* workspace, void* stream);
+
+/* Static English description of a status code (never NULL). */
+const char* mla_status_string(mla_status status);
+
+/* Version of this ABI (major * 10000 + minor * 100 + patch). */
+int32_t mla_decode_abi_version(void);
+
+/*
+ * Test hooks (not for production use).  mla_decode_set_debug() sets
+ * process-wide options applied to subsequent runs:
+ *   wait_timeout_ns  bound of every device pipeline wait (0 = default, 2 s)
+ *   stall_tile       >= 0: the TMA producer of the first CTA skips the load of
+ *                    that pipeline unit while still arming its barrier, so the
+ *                    consumer's bounded wait runs out (exercises the timeout
+ *                    path without faulting or hanging the GPU); -1 = off
+ */
+mla_status mla_decode_set_debug(uint64_t wait_timeout_ns, int32_t stall_tile);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_DECODE_H_ */

@@ -1,0 +1,600 @@
+// kernel_transposed.cuh -- MLA decode main kernel, "transposed" orientation.
+//
+// One CTA handles G query rows (token, head pairs) of one sequence over one
+// contiguous range of its KV tiles.  Per 128-row KV tile:
+//
+//   S^T[128 kv, G] = K_tile[128, 576] . Q_g^T       tcgen05.mma M=128 N=G K=576
+//   softmax over the kv axis (TMEM lanes) in fp32, base 2, lazily rescaled
+//   O^T[512, G]   += V_tile^T[512, 128] . P^T        4 x tcgen05.mma M=128 N=G K=128
+//
+// This is the pages' two-GEMM dataflow ("TileLang: Bridging Programmability and
+// Performance in Modern Neural Kernels", papernotes.org, section "一个完整示例：
+// FlashMLA 的两阶段优化": Q and the KV tile staged in shared memory, S produced
+// by the first GEMM, cast, and fed to the second) re-laid out for sm_100a: the
+// accumulators live in tensor memory, the kv rows sit on the 128 TMEM lanes so
+// that a small number of query rows (G = 16 or 32) still fills an M=128 MMA,
+// and V is read in place as the first 512 columns of the very tile K came in
+// (no second load).  The pipeline is warp specialised ("TileLang 完整解析",
+// section "三大核心優化機制": a TMA producer warp and consumer warps joined by
+// mbarriers), with one warp issuing all tcgen05 MMAs.
+//
+// Warp roles (192 threads):
+//   warps 0-3  softmax + epilogue (thread = TMEM lane = kv row / dv row)
+//   warp 4     TMA producer (one elected lane)
+//   warp 5     TMEM allocator + MMA issuer (one elected lane)
+//
+// Shared memory (1024-byte aligned regions, 128-byte swizzle for TMA data):
+//   pair ring  NP x 32 KB: a [128 kv x 128 col] block = dv chunks 2p, 2p+1
+//   rope ring  NR x 16 KB: the [128 kv x 64] rope chunk (columns 512..575)
+//   Q          9 x [G x 64] chunks, loaded once per piece
+//   P^T        [128 kv x G] bf16, MN-major (q contiguous), 32/64-byte swizzle
+// Every pipeline wait is bounded (%globaltimer); on expiry the CTA records
+// kStatusTimeout, drains its own TMA loads and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace mla {
+
+struct MainArgs {
+    const int32_t* seqlens;
+    int B;
+    int R;            // query rows per sequence (Sq * H)
+    int L_max;
+    int P;            // partitions
+    int NG;           // query-row groups per partition (CTAs sharing a partition)
+    float scale_log2; // softmax_scale * log2(e)
+    __nv_bfloat16* out;
+    float* lse;
+    float* part_o;    // [2P, R, 512]
+    float* part_lse;  // [2P, R]
+    uint32_t* status;
+    unsigned long long timeout_ns;
+    int stall_unit;   // test hook: skip this TMA unit in CTA 0 (-1 = off)
+};
+
+template <int G>
+struct TransposedCfg {
+    static_assert(G == 16 || G == 32, "query rows per CTA");
+    static constexpr int kThreads = 192;
+    static constexpr int NP = (G == 16) ? 5 : 4;  // pair slots (a tile needs 4)
+    static constexpr int NR = 2;                  // rope slots
+    static constexpr int kPairBytes = kTileKV * 128 * 2;     // 32 KB
+    static constexpr int kChunkBytes = kTileKV * 128;        // 16 KB
+    static constexpr int kQChunkBytes = G * 128;
+    static constexpr int kPTBytes = kTileKV * G * 2;
+    static constexpr int OFF_PAIR = 0;
+    static constexpr int OFF_ROPE = OFF_PAIR + NP * kPairBytes;
+    static constexpr int OFF_Q = OFF_ROPE + NR * kChunkBytes;
+    static constexpr int OFF_PT = OFF_Q + kNumChunks * kQChunkBytes;
+    static constexpr int OFF_RED = OFF_PT + kPTBytes;              // floats: [2][4][G] max, [4][G] sums
+    static constexpr int kRedFloats = 12 * G;
+    static constexpr int OFF_BAR = OFF_RED + kRedFloats * 4;
+    // barriers: q_full, q_empty, s_full, p_full, pv_done, drain, group_sync, pair_full[NP],
+    //           pair_empty[NP], rope_full[NR], rope_empty[NR]
+    static constexpr int kNumBars = 7 + 2 * NP + 2 * NR;
+    static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
+    static constexpr int kSmemBytes = OFF_MISC + 64 + 1024;  // + slack to align the base to 1024
+    // TMEM: O^T blocks at columns [0, 4G), S^T at [4G, 5G)
+    static constexpr uint32_t kTmemCols = (5 * G <= 128) ? 128 : 256;
+    static constexpr uint32_t kColS = 4 * G;
+    // P^T swizzle: one row of G bf16 = 2G bytes (32 or 64)
+    static constexpr ptx::Swizzle kPTSwz = (G == 16) ? ptx::Swizzle::B32 : ptx::Swizzle::B64;
+    static constexpr uint32_t kPTAtom = 8 * 2 * G;  // 8 rows x row bytes
+    static constexpr uint32_t kIdescS = ptx::make_idesc_bf16(128, G, 0, 0);
+    static constexpr uint32_t kIdescPV = ptx::make_idesc_bf16(128, G, 1, 1);
+};
+
+// Byte offset of 16-byte unit u of row r in a swizzled region whose rows are
+// `row_bytes` long (32, 64 or 128) -- the XOR pattern TMA and the UMMA
+// descriptors use: unit index ^= (address bits [7, 7+log2(row_bytes/16))).
+__device__ __forceinline__ uint32_t swz_offset(uint32_t r, uint32_t u, uint32_t row_bytes) {
+    const uint32_t addr = r * row_bytes + u * 16;
+    const uint32_t mask = (row_bytes / 16) - 1;
+    return addr ^ (((addr >> 7) & mask) << 4);
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Warp reduce-scatter: v[0..G) per lane -> on return, every lane holds the
+// reduction over the 32 lanes of column col_of_lane(lane) in its return value.
+template <int G, bool kMax>
+__device__ __forceinline__ float warp_reduce_scatter(const float (&v_in)[G], int lane) {
+    constexpr int LOG2G = (G == 16) ? 4 : 5;
+    float v[G];
+#pragma unroll
+    for (int i = 0; i < G; ++i) v[i] = v_in[i];
+#pragma unroll
+    for (int s = 0; s < LOG2G; ++s) {
+        const int h = G >> (s + 1);
+        const int mask = 16 >> s;
+        const bool upper = (lane & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = upper ? v[i] : v[i + h];
+            const float keep = upper ? v[i + h] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, mask);
+            v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+#pragma unroll
+    for (int m = (16 >> LOG2G); m >= 1; m >>= 1) {
+        const float recv = __shfl_xor_sync(0xffffffffu, v[0], m);
+        v[0] = kMax ? fmaxf(v[0], recv) : v[0] + recv;
+    }
+    return v[0];
+}
+
+template <int G>
+__device__ __forceinline__ int col_of_lane(int lane) {
+    return (G == 32) ? lane : (lane >> 1);
+}
+
+template <int G>
+__global__ void __launch_bounds__(192, 1)
+    mla_decode_transposed_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                                 const MainArgs args) {
+    using C = TransposedCfg<G>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    uint8_t* pair_smem = smem + C::OFF_PAIR;
+    uint8_t* rope_smem = smem + C::OFF_ROPE;
+    uint8_t* q_smem = smem + C::OFF_Q;
+    uint8_t* pt_smem = smem + C::OFF_PT;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars + 0;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* s_full = bars + 2;
+    uint64_t* p_full = bars + 3;
+    uint64_t* pv_done = bars + 4;
+    uint64_t* drain = bars + 5;
+    uint64_t* group_sync = bars + 6;  // the 128 softmax threads (bounded, unlike bar.sync)
+    uint64_t* pair_full = bars + 7;
+    uint64_t* pair_empty = pair_full + C::NP;
+    uint64_t* rope_full = pair_empty + C::NP;
+    uint64_t* rope_empty = rope_full + C::NR;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    uint32_t* tmem_base_slot = misc + 0;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+    int* b_first_slot = reinterpret_cast<int*>(misc + 2);
+    long long* acc_first_slot = reinterpret_cast<long long*>(misc + 4);
+    long long* total_slot = reinterpret_cast<long long*>(misc + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int p = blockIdx.x / args.NG;  // partition
+    const int g = blockIdx.x % args.NG;  // query-row group within the sequence
+
+    // ---------------------------------------------------------------- setup
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(q_full, 1);
+        ptx::mbar_init(q_empty, 1);
+        ptx::mbar_init(s_full, 1);
+        ptx::mbar_init(p_full, 128);
+        ptx::mbar_init(pv_done, 1);
+        ptx::mbar_init(drain, 1);
+        ptx::mbar_init(group_sync, 128);
+        for (int i = 0; i < C::NP; ++i) {
+            ptx::mbar_init(pair_full + i, 1);
+            ptx::mbar_init(pair_empty + i, 1);
+        }
+        for (int i = 0; i < C::NR; ++i) {
+            ptx::mbar_init(rope_full + i, 1);
+            ptx::mbar_init(rope_empty + i, 1);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbarrier_init();
+    }
+    if (warp == 5) {
+        ptx::tmem_alloc<C::kTmemCols>(tmem_base_slot);
+        ptx::tmem_relinquish();
+    }
+    if (warp == 0) {
+        // partition bounds in the flat tile space, and the first sequence
+        const long long total = total_tiles_warp(args.seqlens, args.B, args.L_max);
+        const long long T = (total + args.P - 1) / args.P;
+        const long long start = static_cast<long long>(p) * T;
+        int bf;
+        long long af;
+        locate_warp(args.seqlens, args.B, args.L_max, start, &bf, &af);
+        if (lane == 0) {
+            *b_first_slot = bf;
+            *acc_first_slot = af;
+            *total_slot = total;
+        }
+        // flag out-of-range lengths once (partition 0, group 0 only)
+        if (blockIdx.x == 0)
+            for (int b = lane; b < args.B; b += 32) clamp_len(args.seqlens[b], args.L_max, args.status);
+    }
+    if (warp == 4 && lane == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_kv);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_slot;
+
+    PieceWalker walker;
+    {
+        const long long total = *total_slot;
+        const long long T = (total + args.P - 1) / args.P;
+        walker.seqlens = args.seqlens;
+        walker.B = args.B;
+        walker.L_max = args.L_max;
+        walker.p = p;
+        walker.start = static_cast<long long>(p) * T;
+        walker.end = walker.start + T < total ? walker.start + T : total;
+        walker.b = *b_first_slot;
+        walker.acc = *acc_first_slot;
+    }
+    const uint64_t tmo = args.timeout_ns;
+
+    if (warp == 4) {
+        // ============================================================ TMA producer
+        if (ptx::elect_one()) {
+            uint32_t pair_cnt = 0, rope_cnt = 0, piece_cnt = 0;
+            int unit = 0;
+            bool ok = true;
+            // last armed phase per slot, for the drain on abort
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                // Q rows of this group: flattened [B*R, 576] rows b*R + g*G ...
+                if (piece_cnt > 0) ok = ptx::mbar_wait_bounded(q_empty, (piece_cnt - 1) & 1, tmo);
+                if (!ok) break;
+                ptx::mbar_arrive_expect_tx(q_full, kNumChunks * C::kQChunkBytes);
+                const int qrow = pc.b * args.R + g * G;
+                if (!(blockIdx.x == 0 && unit == args.stall_unit))
+                    for (int c = 0; c < kNumChunks; ++c)
+                        ptx::tma_load_2d(q_smem + c * C::kQChunkBytes, &tm_q, q_full, c * kChunk, qrow);
+                ++unit;
+                for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    int row0 = t * kTileKV;
+                    if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;  // end-aligned last tile
+                    {
+                        const uint32_t s = rope_cnt % C::NR;
+                        ok = ptx::mbar_wait_bounded(rope_empty + s, ((rope_cnt / C::NR) & 1) ^ 1, tmo);
+                        if (!ok) break;
+                        ptx::mbar_arrive_expect_tx(rope_full + s, C::kChunkBytes);
+                        if (!(blockIdx.x == 0 && unit == args.stall_unit))
+                            ptx::tma_load_3d(rope_smem + s * C::kChunkBytes, &tm_kv, rope_full + s, 8 * kChunk,
+                                             row0, pc.b);
+                        ++unit;
+                        ++rope_cnt;
+                    }
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const uint32_t s = pair_cnt % C::NP;
+                        ok = ptx::mbar_wait_bounded(pair_empty + s, ((pair_cnt / C::NP) & 1) ^ 1, tmo);
+                        if (!ok) break;
+                        ptx::mbar_arrive_expect_tx(pair_full + s, C::kPairBytes);
+                        if (!(blockIdx.x == 0 && unit == args.stall_unit)) {
+                            uint8_t* dst = pair_smem + s * C::kPairBytes;
+                            ptx::tma_load_3d(dst, &tm_kv, pair_full + s, (2 * pp) * kChunk, row0, pc.b);
+                            ptx::tma_load_3d(dst + C::kChunkBytes, &tm_kv, pair_full + s, (2 * pp + 1) * kChunk,
+                                             row0, pc.b);
+                        }
+                        ++unit;
+                        ++pair_cnt;
+                    }
+                }
+                ++piece_cnt;
+            }
+            if (!ok) {
+                atomicOr(args.status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+            // Drain: every load this thread armed must have landed before the
+            // CTA can exit (bounded; a load that was never issued -- the test
+            // stall -- just runs the bound out).
+            if (piece_cnt > 0 || pair_cnt > 0) {
+                if (piece_cnt > 0) ptx::mbar_wait_bounded(q_full, (piece_cnt - 1) & 1, tmo);
+                for (uint32_t i = 0; i < C::NP && i < pair_cnt; ++i) {
+                    const uint32_t use = pair_cnt - 1 - i;  // the last use of slot use % NP
+                    ptx::mbar_wait_bounded(pair_full + (use % C::NP), (use / C::NP) & 1, tmo);
+                }
+                for (uint32_t i = 0; i < C::NR && i < rope_cnt; ++i) {
+                    const uint32_t use = rope_cnt - 1 - i;
+                    ptx::mbar_wait_bounded(rope_full + (use % C::NR), (use / C::NR) & 1, tmo);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ============================================================ MMA issuer
+        if (ptx::elect_one()) {
+            uint32_t pair_cnt = 0, rope_cnt = 0, piece_cnt = 0, tile_cnt = 0;
+            bool ok = true;
+            const uint32_t q_base = ptx::smem_u32(q_smem);
+            const uint32_t pt_base = ptx::smem_u32(pt_smem);
+            const uint32_t tm_S = tmem_base + C::kColS;
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                for (int t = pc.tile_lo; t < pc.tile_hi; ++t) {
+                    const bool first = (t == pc.tile_lo);
+                    const bool last = (t == pc.tile_hi - 1);
+                    if (first) {
+                        ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
+                        if (!ok) break;
+                    }
+                    // ---------------- S^T = K . Q^T  (rope chunk first, then the 8 value chunks)
+                    const uint32_t rs = rope_cnt % C::NR;
+                    ok = ptx::mbar_wait_bounded(rope_full + rs, (rope_cnt / C::NR) & 1, tmo);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    {
+                        const uint32_t a0 = ptx::smem_u32(rope_smem + rs * C::kChunkBytes);
+                        const uint32_t b0 = q_base + 8 * C::kQChunkBytes;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t da = ptx::make_smem_desc(a0 + kk * 32, 16, 1024, ptx::Swizzle::B128);
+                            const uint64_t db = ptx::make_smem_desc(b0 + kk * 32, 16, 1024, ptx::Swizzle::B128);
+                            ptx::mma_bf16_ss(tm_S, da, db, C::kIdescS, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    ptx::mma_commit(rope_empty + rs);
+                    ++rope_cnt;
+                    uint32_t slots[4];
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const uint32_t s = (pair_cnt + pp) % C::NP;
+                        slots[pp] = s;
+                        ok = ptx::mbar_wait_bounded(pair_full + s, ((pair_cnt + pp) / C::NP) & 1, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        const uint32_t pbase = ptx::smem_u32(pair_smem + s * C::kPairBytes);
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int c = 2 * pp + h;
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint64_t da = ptx::make_smem_desc(pbase + h * C::kChunkBytes + kk * 32, 16,
+                                                                        1024, ptx::Swizzle::B128);
+                                const uint64_t db = ptx::make_smem_desc(q_base + c * C::kQChunkBytes + kk * 32, 16,
+                                                                        1024, ptx::Swizzle::B128);
+                                ptx::mma_bf16_ss(tm_S, da, db, C::kIdescS, 1u);
+                            }
+                        }
+                    }
+                    if (!ok) break;
+                    if (last) ptx::mma_commit(q_empty);
+                    ptx::mma_commit(s_full);
+                    // ---------------- O^T += V^T . P^T  (after the softmax wrote P^T)
+                    ok = ptx::mbar_wait_bounded(p_full, tile_cnt & 1, tmo);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const uint32_t vbase = ptx::smem_u32(pair_smem + slots[pp] * C::kPairBytes);
+                        const uint32_t tm_O = tmem_base + pp * G;
+#pragma unroll
+                        for (int kk = 0; kk < kTileKV / 16; ++kk) {
+                            // A = V^T block: M = 128 dv (two 64-wide atoms 16 KB apart), K = 16 kv rows
+                            const uint64_t da =
+                                ptx::make_smem_desc(vbase + kk * 2048, C::kChunkBytes, 1024, ptx::Swizzle::B128);
+                            // B = P^T: K = 16 kv rows (two 8-row atoms), N = G (one atom wide)
+                            const uint64_t db = ptx::make_smem_desc(pt_base + kk * 2 * C::kPTAtom, C::kPTBytes,
+                                                                    C::kPTAtom, C::kPTSwz);
+                            ptx::mma_bf16_ss(tm_O, da, db, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
+                        }
+                        ptx::mma_commit(pair_empty + slots[pp]);
+                    }
+                    pair_cnt += 4;
+                    if (last) ptx::mma_commit(pv_done);
+                    ++tile_cnt;
+                }
+                ++piece_cnt;
+            }
+            if (!ok) {
+                atomicOr(args.status, kStatusTimeout);
+                *abort_flag = 1;
+            }
+            // drain: all MMAs this thread issued must complete before TMEM is freed
+            ptx::mma_commit(drain);
+            ptx::mbar_wait_bounded(drain, 0, tmo);
+        }
+        __syncwarp();
+    } else {
+        // ============================================================ softmax + epilogue (warps 0-3)
+        const int row_in_tile = warp * 32 + lane;            // TMEM lane = kv row (S^T) = dv row (O^T)
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        const int my_col = col_of_lane<G>(lane);
+        const bool writes_col = (G == 32) || ((lane & 1) == 0);
+        uint32_t tile_cnt = 0, piece_cnt = 0, sync_cnt = 0;
+        bool ok = true;
+        // bounded barrier over the 128 softmax threads
+        auto group_barrier = [&]() -> bool {
+            ptx::mbar_arrive(group_sync);
+            const bool r = ptx::mbar_wait_bounded(group_sync, sync_cnt & 1, tmo);
+            ++sync_cnt;
+            return r;
+        };
+        Piece pc;
+        while (ok && walker.next(pc)) {
+            float m_ref[G];
+            float l_part[G];
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                m_ref[j] = -INFINITY;
+                l_part[j] = 0.f;
+            }
+            for (int t = pc.tile_lo; t < pc.tile_hi; ++t) {
+                const bool first = (t == pc.tile_lo);
+                int row0 = t * kTileKV;
+                if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
+                const int kv_row = row0 + row_in_tile;
+                const bool valid = (kv_row >= t * kTileKV) && (kv_row < pc.L);
+
+                ok = ptx::mbar_wait_bounded(s_full, tile_cnt & 1, tmo);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                float x[G];
+                {
+                    uint32_t r[16];
+#pragma unroll
+                    for (int c0 = 0; c0 < G; c0 += 16) {
+                        ptx::tmem_ld_16(lane_addr + C::kColS + c0, r);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            x[c0 + j] = valid ? __uint_as_float(r[j]) * args.scale_log2 : -INFINITY;
+                    }
+                }
+                // column max over the tile's 128 kv rows
+                float* redmax = red + (tile_cnt & 1) * 4 * G;
+                const float wmax = warp_reduce_scatter<G, true>(x, lane);
+                if (writes_col) redmax[warp * G + my_col] = wmax;
+                ok = group_barrier();
+                if (!ok) break;
+                float tmax[G];
+#pragma unroll
+                for (int j = 0; j < G; j += 4) {
+                    float4 a = *reinterpret_cast<const float4*>(redmax + 0 * G + j);
+                    const float4 b1 = *reinterpret_cast<const float4*>(redmax + 1 * G + j);
+                    const float4 b2 = *reinterpret_cast<const float4*>(redmax + 2 * G + j);
+                    const float4 b3 = *reinterpret_cast<const float4*>(redmax + 3 * G + j);
+                    tmax[j + 0] = fmaxf(fmaxf(a.x, b1.x), fmaxf(b2.x, b3.x));
+                    tmax[j + 1] = fmaxf(fmaxf(a.y, b1.y), fmaxf(b2.y, b3.y));
+                    tmax[j + 2] = fmaxf(fmaxf(a.z, b1.z), fmaxf(b2.z, b3.z));
+                    tmax[j + 3] = fmaxf(fmaxf(a.w, b1.w), fmaxf(b2.w, b3.w));
+                }
+                // Lazy rescale: keep the reference max unless some column grew
+                // by more than 8 (p <= 2^8 then); the decision is identical in
+                // every thread (same shared data), so the branch is uniform.
+                bool grow = false;
+#pragma unroll
+                for (int j = 0; j < G; ++j) grow |= (tmax[j] > m_ref[j] + 8.f);
+                if (first) {
+#pragma unroll
+                    for (int j = 0; j < G; ++j) m_ref[j] = tmax[j];
+                } else if (grow) {
+                    float alpha[G];
+#pragma unroll
+                    for (int j = 0; j < G; ++j) {
+                        const float mn = fmaxf(m_ref[j], tmax[j]);
+                        alpha[j] = ex2_approx(m_ref[j] - mn);
+                        m_ref[j] = mn;
+                        l_part[j] *= alpha[j];
+                    }
+                    // O^T columns j *= alpha[j]; PV of the previous tile has
+                    // completed (it was committed before this tile's S^T).
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) {
+#pragma unroll
+                        for (int c0 = 0; c0 < G; c0 += 16) {
+                            uint32_t r[16];
+                            ptx::tmem_ld_16(lane_addr + blk * G + c0, r);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha[c0 + j]);
+                            ptx::tmem_st_16(lane_addr + blk * G + c0, r);
+                        }
+                    }
+                    ptx::tmem_wait_st();
+                }
+                // P^T row for this kv row: G bf16 values, swizzled MN-major
+                uint32_t packed[G / 2];
+#pragma unroll
+                for (int j = 0; j < G; j += 2) {
+                    const float p0 = ex2_approx(x[j] - m_ref[j]);
+                    const float p1 = ex2_approx(x[j + 1] - m_ref[j + 1]);
+                    l_part[j] += p0;
+                    l_part[j + 1] += p1;
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    packed[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+#pragma unroll
+                for (int u = 0; u < (2 * G) / 16; ++u) {
+                    const uint32_t off = swz_offset(row_in_tile, u, 2 * G);
+                    *reinterpret_cast<uint4*>(pt_smem + off) =
+                        make_uint4(packed[4 * u + 0], packed[4 * u + 1], packed[4 * u + 2], packed[4 * u + 3]);
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(p_full);
+                ++tile_cnt;
+            }
+            if (!ok) break;
+            // ---------------- epilogue: O / l -> out (or a partial), lse
+            ok = ptx::mbar_wait_bounded(pv_done, piece_cnt & 1, tmo);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            float* redsum = red + 8 * G;
+            {
+                const float ws = warp_reduce_scatter<G, false>(l_part, lane);
+                if (writes_col) redsum[warp * G + my_col] = ws;
+            }
+            ok = group_barrier();
+            if (!ok) break;
+            float inv_l[G];
+#pragma unroll
+            for (int j = 0; j < G; ++j)
+                inv_l[j] = 1.f / (redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j]);
+            const int row_base = g * G;  // first query row of this group within the sequence
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) {
+                const int dv = blk * 128 + row_in_tile;
+#pragma unroll
+                for (int c0 = 0; c0 < G; c0 += 16) {
+                    uint32_t r[16];
+                    ptx::tmem_ld_16(lane_addr + blk * G + c0, r);
+                    ptx::tmem_wait_ld();
+                    if (pc.slot < 0) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const size_t orow = static_cast<size_t>(pc.b) * args.R + row_base + c0 + j;
+                            args.out[orow * kDv + dv] = __float2bfloat16_rn(__uint_as_float(r[j]) * inv_l[c0 + j]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const size_t orow = static_cast<size_t>(pc.slot) * args.R + row_base + c0 + j;
+                            args.part_o[orow * kDv + dv] = __uint_as_float(r[j]) * inv_l[c0 + j];
+                        }
+                    }
+                }
+            }
+            if (row_in_tile < G) {
+                const int j = row_in_tile;
+                float mj = 0.f, lj = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < G; ++jj)
+                    if (jj == j) {
+                        mj = m_ref[jj];
+                    }
+                lj = redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j];
+                const float lse_nat = (mj + log2f(lj)) * 0.69314718055994530942f;
+                if (pc.slot < 0)
+                    args.lse[static_cast<size_t>(pc.b) * args.R + row_base + j] = lse_nat;
+                else
+                    args.part_lse[static_cast<size_t>(pc.slot) * args.R + row_base + j] = lse_nat;
+            }
+            ptx::tc_fence_before();
+            // the next piece reuses the sums buffer only after everyone read it
+            ok = group_barrier();
+            ++piece_cnt;
+        }
+        if (!ok) {
+            atomicOr(args.status, kStatusTimeout);
+            *abort_flag = 1;
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc<C::kTmemCols>(tmem_base);
+    }
+}
+
+}  // namespace mla

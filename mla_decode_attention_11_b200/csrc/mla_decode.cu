@@ -1,0 +1,297 @@
+// mla_decode.cu -- host side of the C ABI declared in include/mla_decode.h:
+// argument validation, plan selection, TMA descriptor encoding and kernel
+// launches.  The device code lives in the kernel_*.cuh headers.
+//
+// The driver entry point for TMA descriptors (cuTensorMapEncodeTiled) is
+// fetched through the runtime (cudaGetDriverEntryPoint), so the library links
+// the CUDA runtime statically and does not link libcuda directly: it loads on
+// machines without a GPU driver (symbol checks), and fails with MLA_ERR_CUDA
+// only when a call actually needs the device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mla_decode.h"
+#include "kernel_combine.cuh"
+#include "kernel_transposed.cuh"
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;     // workspace status words
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s
+
+std::atomic<unsigned long long> g_timeout_ns{0};
+std::atomic<int> g_stall_unit{-1};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+struct Layout {
+    size_t part_lse_off, part_o_off, total;
+};
+
+Layout workspace_layout(int P, int R) {
+    Layout l;
+    l.part_lse_off = kHeaderBytes;
+    l.part_o_off = align_up(l.part_lse_off + size_t(2) * P * R * sizeof(float), 256);
+    l.total = l.part_o_off + size_t(2) * P * R * mla::kDv * sizeof(float);
+    return l;
+}
+
+template <int G>
+mla_status launch_transposed(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
+                             const mla::MainArgs& args, cudaStream_t stream) {
+    using C = mla::TransposedCfg<G>;
+    auto kern = mla::mla_decode_transposed_kernel<G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(plan.num_partitions * plan.num_groups));
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, args);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int choose_group_rows(int R) {
+    if (R == 16) return 16;
+    return (R % 32 == 0) ? 32 : 16;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t mla_decode_abi_version(void) { return 10000; }
+
+const char* mla_status_string(mla_status s) {
+    switch (s) {
+        case MLA_OK: return "ok";
+        case MLA_ERR_INVALID_ARG: return "invalid argument";
+        case MLA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case MLA_ERR_UNSUPPORTED: return "unsupported shape or device (needs sm_100)";
+        case MLA_ERR_CUDA: return "CUDA call failed";
+        case MLA_ERR_TIMEOUT: return "device pipeline wait timed out; results invalid";
+        case MLA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MLA_ERR_SEQLEN: return "a sequence length was outside [0, L_max] (clamped)";
+    }
+    return "unknown status";
+}
+
+mla_status mla_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                           int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes) {
+    if (!plan) return MLA_ERR_INVALID_ARG;
+    if (B < 1 || B > 65535 || Sq < 1 || Sq > 16 || L_max < 1 || L_max > (1 << 24)) return MLA_ERR_INVALID_ARG;
+    if (H != 16 && H != 32 && H != 64 && H != 128) return MLA_ERR_UNSUPPORTED;
+    if (num_partitions_override < 0) return MLA_ERR_INVALID_ARG;
+    int sms = 148;  // device < 0: plan for a B200 without touching a device
+    if (device >= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+            cudaGetLastError();
+            return MLA_ERR_CUDA;
+        }
+    }
+    mla_plan p;
+    std::memset(&p, 0, sizeof p);
+    p.B = B;
+    p.Sq = Sq;
+    p.H = H;
+    p.L_max = L_max;
+    p.device = device;
+    p.num_sms = sms;
+    const int R = Sq * H;
+    const int G = choose_group_rows(R);
+    p.kernel = MLA_KERNEL_TRANSPOSED;
+    p.group_rows = G;
+    p.num_groups = R / G;
+    int P = num_partitions_override > 0 ? num_partitions_override : sms / p.num_groups;
+    if (P < 1) P = 1;
+    if (P > 4096) P = 4096;
+    p.num_partitions = P;
+    p.tile_kv = mla::kTileKV;
+    p.cta_threads = 192;
+    p.smem_bytes = (G == 16) ? mla::TransposedCfg<16>::kSmemBytes : mla::TransposedCfg<32>::kSmemBytes;
+    p.workspace_bytes = workspace_layout(P, R).total;
+    *plan = p;
+    if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
+    return MLA_OK;
+}
+
+mla_status mla_decode_workspace_init(const mla_plan* plan, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!plan || !workspace) return MLA_ERR_INVALID_ARG;
+    if (workspace_bytes < plan->workspace_bytes || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+    if (cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                      float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                      void* stream_, int phases) {
+    if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
+    if (!plan || !q || !kv || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    const mla_plan& pl = *plan;
+    const int R = pl.Sq * pl.H;
+    if (pl.B < 1 || pl.Sq < 1 || pl.H < 1 || pl.L_max < 1 || pl.num_partitions < 1 || pl.num_groups < 1 ||
+        pl.group_rows * pl.num_groups != R || pl.kernel != MLA_KERNEL_TRANSPOSED ||
+        (pl.group_rows != 16 && pl.group_rows != 32))
+        return MLA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4))
+        return MLA_ERR_ALIGNMENT;
+    const Layout lay = workspace_layout(pl.num_partitions, R);
+    if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (pl.device >= 0 && dev != pl.device) return MLA_ERR_INVALID_ARG;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+
+    const int G = pl.group_rows;
+    CUtensorMap tm_q, tm_kv;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(pl.B) * R};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kDqk) * 2};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(mla::kChunk), static_cast<cuuint32_t>(G)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(pl.L_max),
+                                    static_cast<cuuint64_t>(pl.B)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk) * 2,
+                                       static_cast<cuuint64_t>(mla::kDqk) * 2 * pl.L_max};
+        const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), static_cast<cuuint32_t>(mla::kTileKV), 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MLA_ERR_CUDA;
+    }
+
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    mla::MainArgs a;
+    a.seqlens = seqlens;
+    a.B = pl.B;
+    a.R = R;
+    a.L_max = pl.L_max;
+    a.P = pl.num_partitions;
+    a.NG = pl.num_groups;
+    a.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
+    a.part_lse = reinterpret_cast<float*>(ws + lay.part_lse_off);
+    a.status = reinterpret_cast<uint32_t*>(ws);
+    const unsigned long long tmo = g_timeout_ns.load();
+    a.timeout_ns = tmo ? tmo : kDefaultTimeoutNs;
+    a.stall_unit = g_stall_unit.load();
+
+    if (phases & 1) {
+        mla_status st = (G == 16) ? launch_transposed<16>(pl, tm_q, tm_kv, a, stream)
+                                  : launch_transposed<32>(pl, tm_q, tm_kv, a, stream);
+        if (st != MLA_OK) {
+            cudaGetLastError();
+            return st;
+        }
+    }
+    if (!(phases & 2)) return MLA_OK;
+    mla::CombineArgs c;
+    c.seqlens = seqlens;
+    c.B = pl.B;
+    c.R = R;
+    c.L_max = pl.L_max;
+    c.P = pl.num_partitions;
+    c.out = a.out;
+    c.lse = lse;
+    c.part_o = a.part_o;
+    c.part_lse = a.part_lse;
+    const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) /
+                                                                        mla::kCombineRowsPerCta));
+    mla::mla_decode_combine_kernel<<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decode_run(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                          float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+    return run_phases(plan, q, kv, seqlens, softmax_scale, out, lse, workspace, workspace_bytes, stream, 3);
+}
+
+mla_status mla_decode_run_phase(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                                float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                void* stream, int32_t phase) {
+    if (phase != 1 && phase != 2) return MLA_ERR_INVALID_ARG;
+    return run_phases(plan, q, kv, seqlens, softmax_scale, out, lse, workspace, workspace_bytes, stream, phase);
+}
+
+mla_status mla_decode_check(const mla_plan* plan, void* workspace, void* stream) {
+    if (!plan || !workspace) return MLA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    uint32_t st = 0;
+    if (cudaMemcpy(&st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(workspace, 0, sizeof st) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (st & mla::kStatusTimeout) return MLA_ERR_TIMEOUT;
+    if (st & mla::kStatusSeqlen) return MLA_ERR_SEQLEN;
+    return MLA_OK;
+}
+
+mla_status mla_decode_set_debug(uint64_t wait_timeout_ns, int32_t stall_tile) {
+    g_timeout_ns.store(wait_timeout_ns);
+    g_stall_unit.store(stall_tile < 0 ? -1 : stall_tile);
+    return MLA_OK;
+}
+
+}  // extern "C"

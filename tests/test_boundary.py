@@ -1,0 +1,110 @@
+"""C-ABI boundary on the CPU: the library builds, loads without a GPU driver,
+exports every symbol include/mla_decode.h declares, and validates arguments
+(without launching anything)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mla_decode_attention_11_b200 import build as B
+from mla_decode_attention_11_b200 import binding as M
+from mla_decode_attention_11_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                            text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return M.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert "mla_decode_plan" in names and "mla_decode_run" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(M.EXPORTED_SYMBOLS) <= set(names)
+
+
+def test_library_links_no_driver(lib):
+    """The .so must not need libcuda.so at load time: it reaches the driver
+    through the statically linked runtime, so it loads on a GPU-less host."""
+    import subprocess
+    needed = subprocess.run(["readelf", "-d", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    assert "libcuda.so" not in needed
+    assert "libcudart.so" not in needed
+    assert lib.mla_decode_abi_version() == 10000
+
+
+def test_status_strings(lib):
+    for code in range(0, 8):
+        s = M.status_string(code)
+        assert isinstance(s, str) and s
+    assert M.status_string(0) == "ok"
+
+
+@pytest.mark.parametrize("name", sorted(W.WORKLOADS))
+def test_plan_for_each_workload(lib, name):
+    w = W.WORKLOADS[name]
+    p = M.mla_decode_plan(w.B, w.Sq, w.H, w.L, device=-1)
+    R = w.Sq * w.H
+    assert p.group_rows * p.num_groups == R
+    assert p.num_partitions >= 1
+    assert p.num_partitions * p.num_groups <= 148
+    assert p.smem_bytes <= 232448
+    assert p.workspace_bytes >= 256 + 2 * p.num_partitions * R * (512 + 1) * 4
+
+
+def test_plan_override_and_clamp(lib):
+    p = M.mla_decode_plan(4, 1, 16, 100, device=-1, num_partitions=1)
+    assert p.num_partitions == 1
+    p = M.mla_decode_plan(4, 1, 16, 100, device=-1, num_partitions=100000)
+    assert p.num_partitions == 4096
+
+
+@pytest.mark.parametrize("args,code", [
+    ((0, 1, 16, 128), 1), ((70000, 1, 16, 128), 1), ((1, 0, 16, 128), 1), ((1, 17, 16, 128), 1),
+    ((1, 1, 16, 0), 1), ((1, 1, 16, (1 << 24) + 1), 1), ((1, 1, 48, 128), 3), ((1, 1, 8, 128), 3),
+])
+def test_plan_rejects(lib, args, code):
+    with pytest.raises(M.MlaError) as e:
+        M.mla_decode_plan(*args, device=-1)
+    assert e.value.code == code
+
+
+def test_run_rejects_without_launching(lib):
+    """Null pointers, misalignment and a short workspace are refused on the
+    host (no device is touched before these checks)."""
+    p = M.mla_decode_plan(2, 1, 16, 256, device=-1)
+    run = lib.mla_decode_run
+    null = None
+    rc = run(ctypes.byref(p), null, 16, 16, ctypes.c_float(0.04), 16, 16, 256, p.workspace_bytes, null)
+    assert rc == 1
+    rc = run(ctypes.byref(p), 16 + 8, 16, 16, ctypes.c_float(0.04), 16, 16, 256, p.workspace_bytes, null)
+    assert rc == 2
+    rc = run(ctypes.byref(p), 16, 16, 16, ctypes.c_float(0.04), 16, 16, 256, p.workspace_bytes - 1, null)
+    assert rc == 6
+    rc = run(ctypes.byref(p), 16, 16, 16, ctypes.c_float(0.04), 16, 16, 0, p.workspace_bytes, null)
+    assert rc == 6
+    rc = run(ctypes.byref(p), 16, 16, 16, ctypes.c_float(float("nan")), 16, 16, 256, p.workspace_bytes, null)
+    assert rc == 1
+    rc = run(None, 16, 16, 16, ctypes.c_float(0.04), 16, 16, 256, p.workspace_bytes, null)
+    assert rc == 1
+
+
+def test_check_rejects_null(lib):
+    assert lib.mla_decode_check(None, None, None) == 1
