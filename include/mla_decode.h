@@ -110,6 +110,18 @@ mla_status mla_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int3
                            int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
 
 /*
+ * mla_decode_plan_kernel -- mla_decode_plan with an explicit kernel choice:
+ * kernel = 0 (automatic: MLA_KERNEL_PAIR when Sq*H is a multiple of 128, else
+ * MLA_KERNEL_TRANSPOSED), MLA_KERNEL_TRANSPOSED (any supported shape) or
+ * MLA_KERNEL_PAIR (MLA_ERR_UNSUPPORTED unless Sq*H % 128 == 0).  Both kernels
+ * compute the same result; the choice only changes speed.  Other arguments,
+ * outputs and return codes as for mla_decode_plan.
+ */
+mla_status mla_decode_plan_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                                  int32_t num_partitions_override, int32_t kernel, mla_plan* plan,
+                                  size_t* workspace_bytes);
+
+/*
  * mla_decode_workspace_init -- zero the workspace's status words on `stream`
  * (asynchronous cudaMemsetAsync of the header).  Call once per workspace before
  * the first run; mla_decode_check() re-zeroes them after reading.

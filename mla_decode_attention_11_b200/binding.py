@@ -32,7 +32,7 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_ALIGNMENT", 3
 MLA_KERNEL_TRANSPOSED = 1
 MLA_KERNEL_PAIR = 2
 
-EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
+EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
                     "mla_decode_check",
                     "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug")
 
@@ -79,6 +79,9 @@ def load_library(build_if_missing: bool = True):
         lib.mla_decode_plan.restype = c_i32
         lib.mla_decode_plan.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(mla_plan),
                                         ctypes.POINTER(c_sz)]
+        lib.mla_decode_plan_kernel.restype = c_i32
+        lib.mla_decode_plan_kernel.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                               ctypes.POINTER(mla_plan), ctypes.POINTER(c_sz)]
         lib.mla_decode_workspace_init.restype = c_i32
         lib.mla_decode_workspace_init.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_sz, c_vp]
         lib.mla_decode_run.restype = c_i32
@@ -110,15 +113,22 @@ def _stream_handle(stream) -> int:
 
 
 def mla_decode_plan(B: int, Sq: int, H: int, L_max: int, device: Optional[int] = None,
-                    num_partitions: int = 0) -> mla_plan:
+                    num_partitions: int = 0, kernel: int = 0) -> mla_plan:
     """Validate a shape and choose kernel / grid / workspace size.  device=None
-    means the current CUDA device; device=-1 plans for a B200 without a GPU."""
+    means the current CUDA device; device=-1 plans for a B200 without a GPU.
+    kernel: 0 = automatic, MLA_KERNEL_TRANSPOSED or MLA_KERNEL_PAIR
+    (mla_decode_plan_kernel)."""
     if device is None:
         device = torch.cuda.current_device()
     p = mla_plan()
     ws = ctypes.c_size_t(0)
-    rc = load_library().mla_decode_plan(int(B), int(Sq), int(H), int(L_max), int(device), int(num_partitions),
-                                        ctypes.byref(p), ctypes.byref(ws))
+    lib = load_library()
+    if kernel:
+        rc = lib.mla_decode_plan_kernel(int(B), int(Sq), int(H), int(L_max), int(device), int(num_partitions),
+                                        int(kernel), ctypes.byref(p), ctypes.byref(ws))
+    else:
+        rc = lib.mla_decode_plan(int(B), int(Sq), int(H), int(L_max), int(device), int(num_partitions),
+                                 ctypes.byref(p), ctypes.byref(ws))
     if rc != MLA_OK:
         raise MlaError(rc, "mla_decode_plan")
     return p

@@ -1,0 +1,504 @@
+// kernel_pair.cuh -- MLA decode main kernel for 128-row query groups, on a
+// CTA pair (cluster of 2, tcgen05 cta_group::2).
+//
+// One CTA pair handles 128 query rows (token, head pairs) of one sequence over
+// one contiguous range of its KV tiles; CTA c of the pair owns query rows
+// [64c, 64c + 64).  Per 128-row KV tile, with the pair MMAs (M = 128 = 2 x 64
+// rows, each CTA supplying its half of A and of B from its own shared memory
+// at the same offset, and receiving its 64 rows of D in its own TMEM):
+//
+//   S[128 q, 128 kv] = Q . K^T      K = 576; B half of CTA c = kv rows [64c, 64c+64)
+//   softmax over kv, fp32, base 2, lazily rescaled; P = bf16
+//   O[128 q, 512]   += P . V        2 MMAs of N = 256; B half of CTA c = 128 of the 256 dv
+//
+// This is the two-GEMM dataflow of "TileLang: Bridging Programmability and
+// Performance in Modern Neural Kernels" (papernotes.org, section "一个完整示例：
+// FlashMLA 的两阶段优化": S produced by the first GEMM is partitioned across the
+// workers and gathered again as the operand of the second GEMM).  On sm_100a
+// the partition is the pair: each SM computes S for its 64 query rows against
+// all 128 keys (the pair MMA gathers the other CTA's keys for it) and
+// accumulates O for its 64 rows over all 512 value columns in its TMEM
+// (64 x 512 fp32 = half of TMEM), so one SM never has to hold O for all 128
+// heads.  Query rows, not value columns, are split, so the row max and row
+// sum stay local to one CTA.
+//
+// Shared memory per CTA:
+//   Q half       9 chunks [64 rows x 64 cols], 128-byte swizzle, K-major (A of S)
+//   K ring       NK chunks [64 kv x 64 cols] of this CTA's kv rows (B of S)
+//   V ring       NV slots [128 kv x 128 dv], two 64-column chunks 16 KB apart,
+//                this CTA's 2 x 128 of the 512 value columns (B of PV, MN-major)
+//   P            [64 rows x 128 kv] bf16, K-major (A of PV)
+// The V operand is loaded separately from K: within one pair MMA both CTAs
+// read their B half at the same shared-memory offset, and the pair's two
+// GEMMs split B along different axes (kv rows for S, value columns for PV),
+// so the value rows this CTA owns for S cannot double as its PV operand.
+//
+// Warp roles (224 threads): warps 0-3 softmax + epilogue (thread = TMEM lane),
+// warp 4 Q/K producer, warp 5 V producer, warp 6 TMEM allocator and (in the
+// leader CTA) the single MMA-issuing thread.  Loads of both CTAs are counted on
+// the leader's barriers (2-SM TMA); MMA completion is multicast to both CTAs.
+// Every wait is bounded; on expiry a CTA records kStatusTimeout and unwinds.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "kernel_transposed.cuh"
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace mla {
+
+template <int NK, int NV>
+struct PairCfg {
+    static constexpr int kThreads = 224;
+    static constexpr int kRows = 64;                          // query rows per CTA
+    static constexpr int kQChunk = kRows * 128;               // 8 KB
+    static constexpr int kKChunk = 64 * 128;                  // 8 KB (64 own kv rows)
+    static constexpr int kVChunk = kTileKV * 128;             // 16 KB
+    static constexpr int kVSlot = 2 * kVChunk;                // 32 KB
+    static constexpr int kPChunk = kRows * 128;               // 8 KB
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + kNumChunks * kQChunk;
+    static constexpr int OFF_V = OFF_K + NK * kKChunk;
+    static constexpr int OFF_P = OFF_V + NV * kVSlot;
+    static constexpr int OFF_RED = OFF_P + 2 * kPChunk;        // floats: [2][128] max, [128] sum
+    static constexpr int OFF_BAR = OFF_RED + 384 * 4;
+    // q_full, q_empty, s_full[2], p_full, pv_done, drain, group_sync, k_full[NK], k_empty[NK],
+    // v_full[NV], v_empty[NV]
+    static constexpr int kNumBars = 8 + 2 * NK + 2 * NV;
+    static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
+    static constexpr int kSmemBytes = OFF_MISC + 64;
+    static constexpr uint32_t kTmemCols = 512;                 // O: [0,256), S buffers: 256, 320
+    static constexpr uint32_t kColS = 256;
+    static constexpr uint32_t kIdescS = ptx::make_idesc_bf16(128, 128, 0, 0);
+    static constexpr uint32_t kIdescPV = ptx::make_idesc_bf16(128, 256, 0, 1);
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+template <int NK, int NV>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
+    mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const MainArgs args) {
+    using C = PairCfg<NK, NV>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+
+    uint8_t* q_smem = smem + C::OFF_Q;
+    uint8_t* k_smem = smem + C::OFF_K;
+    uint8_t* v_smem = smem + C::OFF_V;
+    uint8_t* p_smem = smem + C::OFF_P;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* q_full = bars + 0;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* s_full = bars + 2;     // [2]
+    uint64_t* p_full = bars + 4;
+    uint64_t* pv_done = bars + 5;
+    uint64_t* drain = bars + 6;
+    uint64_t* group_sync = bars + 7;
+    uint64_t* k_full = bars + 8;
+    uint64_t* k_empty = k_full + NK;
+    uint64_t* v_full = k_empty + NK;
+    uint64_t* v_empty = v_full + NV;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    uint32_t* tmem_base_slot = misc + 0;
+    int* b_first_slot = reinterpret_cast<int*>(misc + 2);
+    long long* acc_first_slot = reinterpret_cast<long long*>(misc + 4);
+    long long* total_slot = reinterpret_cast<long long*>(misc + 6);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();  // 0 = leader (issues the pair MMAs)
+    const bool leader = (rank == 0);
+    const int pair_id = blockIdx.x >> 1;
+    const int p = pair_id / args.NG;  // partition
+    const int g = pair_id % args.NG;  // 128-row query group within the sequence
+    const uint64_t tmo = args.timeout_ns;
+    // the shared-memory carve-up assumes a 1024-byte aligned base (128-byte swizzle atoms)
+    const bool smem_ok = (ptx::smem_u32(smem) & 1023u) == 0;
+
+    // ---------------------------------------------------------------- setup
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(q_full, 1);
+        ptx::mbar_init(q_empty, 1);
+        ptx::mbar_init(s_full + 0, 1);
+        ptx::mbar_init(s_full + 1, 1);
+        ptx::mbar_init(p_full, 256);  // every softmax thread of both CTAs
+        ptx::mbar_init(pv_done, 1);
+        ptx::mbar_init(drain, 1);
+        ptx::mbar_init(group_sync, 128);
+        for (int i = 0; i < NK; ++i) {
+            ptx::mbar_init(k_full + i, 1);
+            ptx::mbar_init(k_empty + i, 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            ptx::mbar_init(v_full + i, 1);
+            ptx::mbar_init(v_empty + i, 1);
+        }
+        ptx::fence_mbarrier_init();
+        if (!smem_ok) atomicOr(args.status, kStatusTimeout);
+    }
+    if (warp == 6) {
+        ptx::tmem_alloc_pair<C::kTmemCols>(tmem_base_slot);
+        ptx::tmem_relinquish_pair();
+    }
+    if (warp == 0) {
+        const long long total = total_tiles_warp(args.seqlens, args.B, args.L_max);
+        const long long T = (total + args.P - 1) / args.P;
+        int bf;
+        long long af;
+        locate_warp(args.seqlens, args.B, args.L_max, static_cast<long long>(p) * T, &bf, &af);
+        if (lane == 0) {
+            *b_first_slot = bf;
+            *acc_first_slot = af;
+            *total_slot = total;
+        }
+        if (blockIdx.x == 0)
+            for (int b = lane; b < args.B; b += 32) clamp_len(args.seqlens[b], args.L_max, args.status);
+    }
+    if (warp == 4 && lane == 0) {
+        ptx::prefetch_tmap(&tm_q);
+        ptx::prefetch_tmap(&tm_k);
+        ptx::prefetch_tmap(&tm_v);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync_all();  // peer barriers initialised before any cross-CTA signal
+    ptx::tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_slot;
+
+    PieceWalker walker;
+    {
+        const long long total = *total_slot;
+        const long long T = (total + args.P - 1) / args.P;
+        walker.seqlens = args.seqlens;
+        walker.B = args.B;
+        walker.L_max = args.L_max;
+        walker.p = p;
+        walker.start = static_cast<long long>(p) * T;
+        walker.end = walker.start + T < total ? walker.start + T : total;
+        walker.b = smem_ok ? *b_first_slot : args.B;  // misaligned smem: do nothing
+        walker.acc = *acc_first_slot;
+    }
+    // shared::cluster addresses of the leader's barriers
+    const uint32_t lead_q_full = ptx::mapa_shared(ptx::smem_u32(q_full), 0);
+    const uint32_t lead_p_full = ptx::mapa_shared(ptx::smem_u32(p_full), 0);
+    const bool stall_cta = (blockIdx.x == 0);
+
+    if (warp == 4) {
+        // ============================================================ Q + K producer
+        if (ptx::elect_one()) {
+            uint32_t k_cnt = 0, piece_cnt = 0;
+            int unit = 0;
+            bool ok = true;
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                if (piece_cnt > 0) ok = ptx::mbar_wait_bounded(q_empty, (piece_cnt - 1) & 1, tmo);
+                if (!ok) break;
+                if (leader) ptx::mbar_arrive_expect_tx(q_full, 2 * kNumChunks * C::kQChunk);
+                const int qrow = pc.b * args.R + g * 128 + static_cast<int>(rank) * 64;
+                if (!(stall_cta && unit == args.stall_unit))
+                    for (int c = 0; c < kNumChunks; ++c)
+                        ptx::tma_load_2d_pair(q_smem + c * C::kQChunk, &tm_q, lead_q_full, c * kChunk, qrow);
+                ++unit;
+                for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    int row0 = t * kTileKV;
+                    if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
+                    const int krow = row0 + static_cast<int>(rank) * 64;
+                    for (int jj = 0; jj < kNumChunks; ++jj) {
+                        const int j = (jj == 0) ? 8 : jj - 1;  // rope chunk first
+                        const uint32_t s = k_cnt % NK;
+                        ok = ptx::mbar_wait_bounded(k_empty + s, ((k_cnt / NK) & 1) ^ 1, tmo);
+                        if (!ok) break;
+                        if (leader) ptx::mbar_arrive_expect_tx(k_full + s, 2 * C::kKChunk);
+                        if (!(stall_cta && unit == args.stall_unit))
+                            ptx::tma_load_3d_pair(k_smem + s * C::kKChunk, &tm_k,
+                                                  ptx::mapa_shared(ptx::smem_u32(k_full + s), 0), j * kChunk,
+                                                  krow, pc.b);
+                        ++unit;
+                        ++k_cnt;
+                    }
+                }
+                ++piece_cnt;
+            }
+            if (!ok) atomicOr(args.status, kStatusTimeout);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ============================================================ V producer
+        if (ptx::elect_one()) {
+            uint32_t v_cnt = 0;
+            bool ok = true;
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    int row0 = t * kTileKV;
+                    if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
+                    for (int i = 0; i < 2; ++i) {
+                        const uint32_t s = v_cnt % NV;
+                        ok = ptx::mbar_wait_bounded(v_empty + s, ((v_cnt / NV) & 1) ^ 1, tmo);
+                        if (!ok) break;
+                        if (leader) ptx::mbar_arrive_expect_tx(v_full + s, 2 * C::kVSlot);
+                        const int col0 = 256 * i + 128 * static_cast<int>(rank);
+                        uint8_t* dst = v_smem + s * C::kVSlot;
+                        const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(v_full + s), 0);
+                        ptx::tma_load_3d_pair(dst, &tm_v, bar, col0, row0, pc.b);
+                        ptx::tma_load_3d_pair(dst + C::kVChunk, &tm_v, bar, col0 + 64, row0, pc.b);
+                        ++v_cnt;
+                    }
+                }
+            }
+            if (!ok) atomicOr(args.status, kStatusTimeout);
+        }
+        __syncwarp();
+    } else if (warp == 6) {
+        // ============================================================ MMA issuer (leader only)
+        if (leader && ptx::elect_one()) {
+            uint32_t k_cnt = 0, v_cnt = 0, piece_cnt = 0, tile_cnt = 0;
+            bool ok = true;
+            const uint32_t q_base = ptx::smem_u32(q_smem);
+            const uint32_t k_base = ptx::smem_u32(k_smem);
+            const uint32_t v_base = ptx::smem_u32(v_smem);
+            const uint32_t p_base = ptx::smem_u32(p_smem);
+            constexpr uint16_t kBoth = 0x3;
+            // O += P . V for global tile index u
+            auto issue_pv = [&](uint32_t u, bool first_of_piece) -> bool {
+                if (!ptx::mbar_wait_bounded_cluster(p_full, u & 1, tmo)) return false;
+                ptx::tc_fence_after();
+                for (int i = 0; i < 2; ++i) {
+                    const uint32_t s = v_cnt % NV;
+                    if (!ptx::mbar_wait_bounded(v_full + s, (v_cnt / NV) & 1, tmo)) return false;
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTileKV / 16; ++kk) {
+                        const uint64_t da = ptx::make_smem_desc(p_base + (kk >> 2) * C::kPChunk + (kk & 3) * 32, 16,
+                                                                1024, ptx::Swizzle::B128);
+                        const uint64_t db = ptx::make_smem_desc(v_base + s * C::kVSlot + kk * 2048, C::kVChunk, 1024,
+                                                                ptx::Swizzle::B128);
+                        ptx::mma_bf16_ss_pair(tmem_base + 128 * i, da, db, C::kIdescPV,
+                                              (first_of_piece && kk == 0) ? 0u : 1u);
+                    }
+                    ptx::mma_commit_pair_mc(v_empty + s, kBoth);
+                    ++v_cnt;
+                }
+                ptx::mma_commit_pair_mc(pv_done, kBoth);
+                return true;
+            };
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    if (t == pc.tile_lo) {
+                        ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
+                        if (!ok) break;
+                    }
+                    // ---------------- S(t) = Q . K^T into S buffer (tile_cnt & 1)
+                    const uint32_t tm_S = tmem_base + C::kColS + 64 * (tile_cnt & 1);
+                    for (int jj = 0; jj < kNumChunks; ++jj) {
+                        const int j = (jj == 0) ? 8 : jj - 1;
+                        const uint32_t s = k_cnt % NK;
+                        ok = ptx::mbar_wait_bounded(k_full + s, (k_cnt / NK) & 1, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t da = ptx::make_smem_desc(q_base + j * C::kQChunk + kk * 32, 16, 1024,
+                                                                    ptx::Swizzle::B128);
+                            const uint64_t db = ptx::make_smem_desc(k_base + s * C::kKChunk + kk * 32, 16, 1024,
+                                                                    ptx::Swizzle::B128);
+                            ptx::mma_bf16_ss_pair(tm_S, da, db, C::kIdescS, (jj | kk) ? 1u : 0u);
+                        }
+                        ptx::mma_commit_pair_mc(k_empty + s, kBoth);
+                        ++k_cnt;
+                    }
+                    if (!ok) break;
+                    if (t == pc.tile_hi - 1) ptx::mma_commit_pair_mc(q_empty, kBoth);
+                    ptx::mma_commit_pair_mc(s_full + (tile_cnt & 1), kBoth);
+                    // ---------------- PV of the previous tile of this piece
+                    if (t > pc.tile_lo) {
+                        ok = issue_pv(tile_cnt - 1, t - 1 == pc.tile_lo);
+                        if (!ok) break;
+                    }
+                    ++tile_cnt;
+                }
+                if (!ok) break;
+                ok = issue_pv(tile_cnt - 1, pc.tile_hi - 1 == pc.tile_lo);
+                ++piece_cnt;
+            }
+            if (!ok) atomicOr(args.status, kStatusTimeout);
+            // drain: every MMA issued must complete before TMEM is freed
+            ptx::mma_commit_pair_mc(drain, 0x1);
+            ptx::mbar_wait_bounded(drain, 0, tmo);
+        }
+        __syncwarp();
+    } else {
+        // ============================================================ softmax + epilogue (warps 0-3)
+        const int L_id = warp * 32 + lane;  // TMEM lane
+        const int r = L_id & 63;            // query row within this CTA's 64
+        const int h = L_id >> 6;            // which 64 keys of the tile (S), which 128 dv of each N=256 (O)
+        const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+        uint32_t tile_cnt = 0, sync_cnt = 0;
+        bool ok = true;
+        auto group_barrier = [&]() -> bool {
+            ptx::mbar_arrive(group_sync);
+            const bool rr = ptx::mbar_wait_bounded(group_sync, sync_cnt & 1, tmo);
+            ++sync_cnt;
+            return rr;
+        };
+        Piece pc;
+        while (ok && walker.next(pc)) {
+            float m_ref = -INFINITY;
+            float l_part = 0.f;
+            for (int t = pc.tile_lo; t < pc.tile_hi; ++t) {
+                const bool first = (t == pc.tile_lo);
+                int row0 = t * kTileKV;
+                if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
+                const int kv0 = row0 + 64 * h;       // key of column j is kv0 + j
+                const int lo = t * kTileKV;          // keys below lo belong to the previous tile
+                const uint32_t buf = tile_cnt & 1;
+                ok = ptx::mbar_wait_bounded(s_full + buf, (tile_cnt >> 1) & 1, tmo);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                float x[64];
+                {
+                    uint32_t rr[32];
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        ptx::tmem_ld_32(lane_addr + C::kColS + 64 * buf + c0, rr);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int kv = kv0 + c0 + j;
+                            x[c0 + j] = (kv >= lo && kv < pc.L) ? __uint_as_float(rr[j]) * args.scale_log2 : -INFINITY;
+                        }
+                    }
+                }
+                float mloc = x[0];
+#pragma unroll
+                for (int j = 1; j < 64; ++j) mloc = fmaxf(mloc, x[j]);
+                float* redmax = red + (tile_cnt & 1) * 128;
+                redmax[L_id] = mloc;
+                ok = group_barrier();
+                if (!ok) break;
+                const float mrow = fmaxf(mloc, redmax[L_id ^ 64]);
+                if (!first) {
+                    // P and O are free once the previous tile's PV has completed
+                    ok = ptx::mbar_wait_bounded(pv_done, (tile_cnt - 1) & 1, tmo);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                }
+                if (first) {
+                    m_ref = mrow;
+                } else {
+                    // lazy rescale: only when the row max grew by more than 8 (p <= 2^8 otherwise)
+                    const bool grow = mrow > m_ref + 8.f;
+                    if (__any_sync(0xffffffffu, grow)) {
+                        float alpha = 1.f;
+                        if (grow) {
+                            alpha = ex2_approx(m_ref - mrow);
+                            m_ref = mrow;
+                            l_part *= alpha;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+#pragma unroll
+                            for (int c0 = 0; c0 < 128; c0 += 32) {
+                                uint32_t rr[32];
+                                ptx::tmem_ld_32(lane_addr + 128 * i + c0, rr);
+                                ptx::tmem_wait_ld();
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * alpha);
+                                ptx::tmem_st_32(lane_addr + 128 * i + c0, rr);
+                            }
+                        }
+                        ptx::tmem_wait_st();
+                    }
+                }
+                // P[r][64h .. 64h+63] = exp2(x - m_ref) as bf16, K-major 128-byte swizzled
+                uint8_t* prow = p_smem + h * C::kPChunk + r * 128;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float a0 = ex2_approx(x[8 * u + 2 * e] - m_ref);
+                        const float a1 = ex2_approx(x[8 * u + 2 * e + 1] - m_ref);
+                        l_part += a0 + a1;
+                        const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+                        w4[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                    }
+                    *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive_cluster(lead_p_full);
+                ++tile_cnt;
+            }
+            if (!ok) break;
+            // ---------------- epilogue: O / l -> out (or a partial), lse
+            ok = ptx::mbar_wait_bounded(pv_done, (tile_cnt - 1) & 1, tmo);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            float* redsum = red + 256;
+            redsum[L_id] = l_part;
+            ok = group_barrier();
+            if (!ok) break;
+            const float l_row = l_part + redsum[L_id ^ 64];
+            const float inv_l = 1.f / l_row;
+            const int qrow = g * 128 + static_cast<int>(rank) * 64 + r;  // row within the sequence
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t rr[32];
+                    ptx::tmem_ld_32(lane_addr + 128 * i + c0, rr);
+                    ptx::tmem_wait_ld();
+                    const int dv0 = 256 * i + 128 * h + c0;
+                    if (pc.slot < 0) {
+                        __nv_bfloat16* dst = args.out + (static_cast<size_t>(pc.b) * args.R + qrow) * kDv + dv0;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 hv =
+                                    __floats2bfloat162_rn(__uint_as_float(rr[8 * v + 2 * e]) * inv_l,
+                                                          __uint_as_float(rr[8 * v + 2 * e + 1]) * inv_l);
+                                w4[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                            }
+                            *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        }
+                    } else {
+                        float* dst = args.part_o + (static_cast<size_t>(pc.slot) * args.R + qrow) * kDv + dv0;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            *reinterpret_cast<float4*>(dst + 4 * v) =
+                                make_float4(__uint_as_float(rr[4 * v + 0]) * inv_l, __uint_as_float(rr[4 * v + 1]) * inv_l,
+                                            __uint_as_float(rr[4 * v + 2]) * inv_l, __uint_as_float(rr[4 * v + 3]) * inv_l);
+                    }
+                }
+            }
+            if (h == 0) {
+                const float lse_nat = (m_ref + log2f(l_row)) * 0.69314718055994530942f;
+                if (pc.slot < 0)
+                    args.lse[static_cast<size_t>(pc.b) * args.R + qrow] = lse_nat;
+                else
+                    args.part_lse[static_cast<size_t>(pc.slot) * args.R + qrow] = lse_nat;
+            }
+            ptx::tc_fence_before();
+            ok = group_barrier();  // sums buffer reused by the next piece
+        }
+        if (!ok) atomicOr(args.status, kStatusTimeout);
+    }
+
+    // ---------------------------------------------------------------- teardown
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::cluster_sync_all();  // both CTAs finished (the leader drained its MMAs) before freeing TMEM
+    if (warp == 6) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc_pair<C::kTmemCols>(tmem_base);
+    }
+}
+
+}  // namespace mla

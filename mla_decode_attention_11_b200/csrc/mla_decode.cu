@@ -18,6 +18,7 @@
 
 #include "../../include/mla_decode.h"
 #include "kernel_combine.cuh"
+#include "kernel_pair.cuh"
 #include "kernel_transposed.cuh"
 
 namespace {
@@ -78,6 +79,45 @@ int choose_group_rows(int R) {
     return (R % 32 == 0) ? 32 : 16;
 }
 
+// pair-kernel ring depths: K chunks (8 KB each) and V slots (32 KB each)
+constexpr int kPairNK = 5;
+constexpr int kPairNV = 3;
+using PairC = mla::PairCfg<kPairNK, kPairNV>;
+
+mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                       const CUtensorMap& tm_v, const mla::MainArgs& args, cudaStream_t stream) {
+    auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairC::kSmemBytes) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(2 * plan.num_partitions * plan.num_groups));
+    kern<<<grid, PairC::kThreads, PairC::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, args);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+bool encode_2d_bf16(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint32_t box_inner, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// kv viewed as [B][L_max][576]: a box of box_rows rows x 64 columns of one sequence
+bool encode_kv(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int B, uint32_t box_rows) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(L_max),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk) * 2,
+                                   static_cast<cuuint64_t>(mla::kDqk) * 2 * L_max};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -100,7 +140,14 @@ const char* mla_status_string(mla_status s) {
 
 mla_status mla_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
                            int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes) {
+    return mla_decode_plan_kernel(B, Sq, H, L_max, device, num_partitions_override, 0, plan, workspace_bytes);
+}
+
+mla_status mla_decode_plan_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                                  int32_t num_partitions_override, int32_t kernel, mla_plan* plan,
+                                  size_t* workspace_bytes) {
     if (!plan) return MLA_ERR_INVALID_ARG;
+    if (kernel != 0 && kernel != MLA_KERNEL_TRANSPOSED && kernel != MLA_KERNEL_PAIR) return MLA_ERR_INVALID_ARG;
     if (B < 1 || B > 65535 || Sq < 1 || Sq > 16 || L_max < 1 || L_max > (1 << 24)) return MLA_ERR_INVALID_ARG;
     if (H != 16 && H != 32 && H != 64 && H != 128) return MLA_ERR_UNSUPPORTED;
     if (num_partitions_override < 0) return MLA_ERR_INVALID_ARG;
@@ -120,17 +167,29 @@ mla_status mla_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int3
     p.device = device;
     p.num_sms = sms;
     const int R = Sq * H;
-    const int G = choose_group_rows(R);
-    p.kernel = MLA_KERNEL_TRANSPOSED;
-    p.group_rows = G;
-    p.num_groups = R / G;
-    int P = num_partitions_override > 0 ? num_partitions_override : sms / p.num_groups;
+    if (kernel == 0) kernel = (R % 128 == 0) ? MLA_KERNEL_PAIR : MLA_KERNEL_TRANSPOSED;
+    if (kernel == MLA_KERNEL_PAIR && R % 128 != 0) return MLA_ERR_UNSUPPORTED;
+    p.kernel = kernel;
+    int ctas_per_partition;
+    if (kernel == MLA_KERNEL_PAIR) {
+        p.group_rows = 128;
+        p.num_groups = R / 128;
+        p.cta_threads = PairC::kThreads;
+        p.smem_bytes = PairC::kSmemBytes;
+        ctas_per_partition = 2 * p.num_groups;
+    } else {
+        const int G = choose_group_rows(R);
+        p.group_rows = G;
+        p.num_groups = R / G;
+        p.cta_threads = 192;
+        p.smem_bytes = (G == 16) ? mla::TransposedCfg<16>::kSmemBytes : mla::TransposedCfg<32>::kSmemBytes;
+        ctas_per_partition = p.num_groups;
+    }
+    int P = num_partitions_override > 0 ? num_partitions_override : sms / ctas_per_partition;
     if (P < 1) P = 1;
     if (P > 4096) P = 4096;
     p.num_partitions = P;
     p.tile_kv = mla::kTileKV;
-    p.cta_threads = 192;
-    p.smem_bytes = (G == 16) ? mla::TransposedCfg<16>::kSmemBytes : mla::TransposedCfg<32>::kSmemBytes;
     p.workspace_bytes = workspace_layout(P, R).total;
     *plan = p;
     if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
@@ -160,9 +219,15 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     const mla_plan& pl = *plan;
     const int R = pl.Sq * pl.H;
     if (pl.B < 1 || pl.Sq < 1 || pl.H < 1 || pl.L_max < 1 || pl.num_partitions < 1 || pl.num_groups < 1 ||
-        pl.group_rows * pl.num_groups != R || pl.kernel != MLA_KERNEL_TRANSPOSED ||
-        (pl.group_rows != 16 && pl.group_rows != 32))
+        pl.group_rows * pl.num_groups != R)
         return MLA_ERR_INVALID_ARG;
+    if (pl.kernel == MLA_KERNEL_TRANSPOSED) {
+        if (pl.group_rows != 16 && pl.group_rows != 32) return MLA_ERR_INVALID_ARG;
+    } else if (pl.kernel == MLA_KERNEL_PAIR) {
+        if (pl.group_rows != 128) return MLA_ERR_INVALID_ARG;
+    } else {
+        return MLA_ERR_INVALID_ARG;
+    }
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4))
         return MLA_ERR_ALIGNMENT;
     const Layout lay = workspace_layout(pl.num_partitions, R);
@@ -185,27 +250,16 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     if (!enc) return MLA_ERR_CUDA;
 
     const int G = pl.group_rows;
-    CUtensorMap tm_q, tm_kv;
-    {
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(pl.B) * R};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kDqk) * 2};
-        const cuuint32_t box[2] = {static_cast<cuuint32_t>(mla::kChunk), static_cast<cuuint32_t>(G)};
-        const cuuint32_t estr[2] = {1, 1};
-        if (enc(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    CUtensorMap tm_q, tm_kv, tm_k;
+    if (pl.kernel == MLA_KERNEL_PAIR) {
+        // Q: 64-row halves; K: 64 own kv rows per CTA; V: all 128 rows of a tile
+        if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, 64) ||
+            !encode_kv(enc, &tm_k, kv, pl.L_max, pl.B, 64) ||
+            !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV))
             return MLA_ERR_CUDA;
-    }
-    {
-        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(pl.L_max),
-                                    static_cast<cuuint64_t>(pl.B)};
-        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk) * 2,
-                                       static_cast<cuuint64_t>(mla::kDqk) * 2 * pl.L_max};
-        const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), static_cast<cuuint32_t>(mla::kTileKV), 1};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        if (enc(&tm_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    } else {
+        if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, G) ||
+            !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV))
             return MLA_ERR_CUDA;
     }
 
@@ -229,8 +283,12 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     a.stall_unit = g_stall_unit.load();
 
     if (phases & 1) {
-        mla_status st = (G == 16) ? launch_transposed<16>(pl, tm_q, tm_kv, a, stream)
-                                  : launch_transposed<32>(pl, tm_q, tm_kv, a, stream);
+        mla_status st;
+        if (pl.kernel == MLA_KERNEL_PAIR)
+            st = launch_pair(pl, tm_q, tm_k, tm_kv, a, stream);
+        else
+            st = (G == 16) ? launch_transposed<16>(pl, tm_q, tm_kv, a, stream)
+                           : launch_transposed<32>(pl, tm_q, tm_kv, a, stream);
         if (st != MLA_OK) {
             cudaGetLastError();
             return st;
