@@ -81,7 +81,10 @@ typedef struct mla_plan {
     int32_t cta_threads;       /* threads per CTA of the main kernel */
     uint64_t smem_bytes;       /* dynamic shared memory per CTA of the main kernel */
     uint64_t workspace_bytes;  /* bytes the caller must provide to mla_decode_run */
-    uint64_t reserved[6];
+    int32_t l2_prefetch_tiles; /* KV tiles the loader prefetches into L2 ahead of its shared-memory
+                                  loads (0..16; a tuning knob, does not change results) */
+    int32_t reserved32;
+    uint64_t reserved[5];
 } mla_plan;
 
 /*

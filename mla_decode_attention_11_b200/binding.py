@@ -49,10 +49,11 @@ class mla_plan(ctypes.Structure):
                 ("group_rows", ctypes.c_int32), ("num_groups", ctypes.c_int32),
                 ("num_partitions", ctypes.c_int32), ("tile_kv", ctypes.c_int32), ("cta_threads", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
-                ("reserved", ctypes.c_uint64 * 6)]
+                ("l2_prefetch_tiles", ctypes.c_int32), ("reserved32", ctypes.c_int32),
+                ("reserved", ctypes.c_uint64 * 5)]
 
     def as_dict(self):
-        return {k: getattr(self, k) for k, _ in self._fields_ if k != "reserved"}
+        return {k: getattr(self, k) for k, _ in self._fields_ if not k.startswith("reserved")}
 
 
 _lock = threading.Lock()

@@ -50,7 +50,7 @@
 
 namespace mla {
 
-template <int NK, int NV>
+template <int NK, int NV, int NS>
 struct PairCfg {
     static constexpr int kThreads = 224;
     static constexpr int kRows = 64;                          // query rows per CTA
@@ -65,23 +65,24 @@ struct PairCfg {
     static constexpr int OFF_P = OFF_V + NV * kVSlot;
     static constexpr int OFF_RED = OFF_P + 2 * kPChunk;        // floats: [2][128] max, [128] sum
     static constexpr int OFF_BAR = OFF_RED + 384 * 4;
-    // q_full, q_empty, s_full[2], p_full, pv_done, drain, group_sync, k_full[NK], k_empty[NK],
+    // q_full, q_empty, p_full, pv_done, drain, group_sync, s_full[NS], k_full[NK], k_empty[NK],
     // v_full[NV], v_empty[NV]
-    static constexpr int kNumBars = 8 + 2 * NK + 2 * NV;
+    static constexpr int kNumBars = 6 + NS + 2 * NK + 2 * NV;
     static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
     static constexpr int kSmemBytes = OFF_MISC + 64;
-    static constexpr uint32_t kTmemCols = 512;                 // O: [0,256), S buffers: 256, 320
+    static constexpr uint32_t kTmemCols = 512;                 // O: [0,256), S buffers from 256, 64 each
     static constexpr uint32_t kColS = 256;
+    static_assert(NS >= 2 && 256 + 64 * NS <= 512, "S buffers must fit next to O in TMEM");
     static constexpr uint32_t kIdescS = ptx::make_idesc_bf16(128, 128, 0, 0);
     static constexpr uint32_t kIdescPV = ptx::make_idesc_bf16(128, 256, 0, 1);
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-template <int NK, int NV>
+template <int NK, int NV, int NS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const MainArgs args) {
-    using C = PairCfg<NK, NV>;
+    using C = PairCfg<NK, NV, NS>;
     extern __shared__ __align__(1024) uint8_t smem[];
 
     uint8_t* q_smem = smem + C::OFF_Q;
@@ -92,12 +93,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars + 0;
     uint64_t* q_empty = bars + 1;
-    uint64_t* s_full = bars + 2;     // [2]
-    uint64_t* p_full = bars + 4;
-    uint64_t* pv_done = bars + 5;
-    uint64_t* drain = bars + 6;
-    uint64_t* group_sync = bars + 7;
-    uint64_t* k_full = bars + 8;
+    uint64_t* p_full = bars + 2;
+    uint64_t* pv_done = bars + 3;
+    uint64_t* drain = bars + 4;
+    uint64_t* group_sync = bars + 5;
+    uint64_t* s_full = bars + 6;     // [NS]
+    uint64_t* k_full = s_full + NS;
     uint64_t* k_empty = k_full + NK;
     uint64_t* v_full = k_empty + NK;
     uint64_t* v_empty = v_full + NV;
@@ -122,8 +123,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     if (threadIdx.x == 0) {
         ptx::mbar_init(q_full, 1);
         ptx::mbar_init(q_empty, 1);
-        ptx::mbar_init(s_full + 0, 1);
-        ptx::mbar_init(s_full + 1, 1);
+        for (int i = 0; i < NS; ++i) ptx::mbar_init(s_full + i, 1);
         ptx::mbar_init(p_full, 256);  // every softmax thread of both CTAs
         ptx::mbar_init(pv_done, 1);
         ptx::mbar_init(drain, 1);
@@ -230,9 +230,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
         if (ptx::elect_one()) {
             uint32_t v_cnt = 0;
             bool ok = true;
+            const int pf = args.prefetch_tiles;
+            // L2 prefetch of a whole tile, split between the two CTAs by column chunk
+            auto prefetch_tile = [&](const Piece& pc, int t) {
+                int row0 = t * kTileKV;
+                if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
+                for (int j = static_cast<int>(rank); j < kNumChunks; j += 2)
+                    ptx::tma_prefetch_3d(&tm_v, j * kChunk, row0, pc.b);
+            };
             Piece pc;
             while (ok && walker.next(pc)) {
+                for (int t = pc.tile_lo; t < pc.tile_lo + pf && t < pc.tile_hi; ++t) prefetch_tile(pc, t);
                 for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    if (pf > 0 && t + pf < pc.tile_hi) prefetch_tile(pc, t + pf);
                     int row0 = t * kTileKV;
                     if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
                     for (int i = 0; i < 2; ++i) {
@@ -285,44 +295,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
                 ptx::mma_commit_pair_mc(pv_done, kBoth);
                 return true;
             };
+            // S(t) for global tile index u into S buffer u % NS
+            auto issue_s = [&](uint32_t u, bool last_of_piece) -> bool {
+                const uint32_t tm_S = tmem_base + C::kColS + 64 * (u % NS);
+                for (int jj = 0; jj < kNumChunks; ++jj) {
+                    const int j = (jj == 0) ? 8 : jj - 1;  // rope chunk first
+                    const uint32_t s = k_cnt % NK;
+                    if (!ptx::mbar_wait_bounded(k_full + s, (k_cnt / NK) & 1, tmo)) return false;
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t da = ptx::make_smem_desc(q_base + j * C::kQChunk + kk * 32, 16, 1024,
+                                                                ptx::Swizzle::B128);
+                        const uint64_t db = ptx::make_smem_desc(k_base + s * C::kKChunk + kk * 32, 16, 1024,
+                                                                ptx::Swizzle::B128);
+                        ptx::mma_bf16_ss_pair(tm_S, da, db, C::kIdescS, (jj | kk) ? 1u : 0u);
+                    }
+                    ptx::mma_commit_pair_mc(k_empty + s, kBoth);
+                    ++k_cnt;
+                }
+                if (last_of_piece) ptx::mma_commit_pair_mc(q_empty, kBoth);
+                ptx::mma_commit_pair_mc(s_full + (u % NS), kBoth);
+                return true;
+            };
+            // PV trails S by NS-1 tiles, so the softmax of a tile overlaps the
+            // QK^T of the next NS-1 tiles.
+            constexpr int kLag = NS - 1;
             Piece pc;
             while (ok && walker.next(pc)) {
-                for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
-                    if (t == pc.tile_lo) {
-                        ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
-                        if (!ok) break;
-                    }
-                    // ---------------- S(t) = Q . K^T into S buffer (tile_cnt & 1)
-                    const uint32_t tm_S = tmem_base + C::kColS + 64 * (tile_cnt & 1);
-                    for (int jj = 0; jj < kNumChunks; ++jj) {
-                        const int j = (jj == 0) ? 8 : jj - 1;
-                        const uint32_t s = k_cnt % NK;
-                        ok = ptx::mbar_wait_bounded(k_full + s, (k_cnt / NK) & 1, tmo);
-                        if (!ok) break;
-                        ptx::tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t da = ptx::make_smem_desc(q_base + j * C::kQChunk + kk * 32, 16, 1024,
-                                                                    ptx::Swizzle::B128);
-                            const uint64_t db = ptx::make_smem_desc(k_base + s * C::kKChunk + kk * 32, 16, 1024,
-                                                                    ptx::Swizzle::B128);
-                            ptx::mma_bf16_ss_pair(tm_S, da, db, C::kIdescS, (jj | kk) ? 1u : 0u);
-                        }
-                        ptx::mma_commit_pair_mc(k_empty + s, kBoth);
-                        ++k_cnt;
-                    }
-                    if (!ok) break;
-                    if (t == pc.tile_hi - 1) ptx::mma_commit_pair_mc(q_empty, kBoth);
-                    ptx::mma_commit_pair_mc(s_full + (tile_cnt & 1), kBoth);
-                    // ---------------- PV of the previous tile of this piece
-                    if (t > pc.tile_lo) {
-                        ok = issue_pv(tile_cnt - 1, t - 1 == pc.tile_lo);
-                        if (!ok) break;
-                    }
-                    ++tile_cnt;
+                const int n = pc.tile_hi - pc.tile_lo;
+                ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
+                const uint32_t u0 = tile_cnt;  // global index of the piece's first tile
+                for (int i = 0; ok && i < n + kLag; ++i) {
+                    if (i < n) ok = issue_s(u0 + i, i == n - 1);
+                    if (ok && i >= kLag) ok = issue_pv(u0 + i - kLag, i - kLag == 0);
                 }
-                if (!ok) break;
-                ok = issue_pv(tile_cnt - 1, pc.tile_hi - 1 == pc.tile_lo);
+                tile_cnt += n;
                 ++piece_cnt;
             }
             if (!ok) atomicOr(args.status, kStatusTimeout);
@@ -355,8 +363,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
                 if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
                 const int kv0 = row0 + 64 * h;       // key of column j is kv0 + j
                 const int lo = t * kTileKV;          // keys below lo belong to the previous tile
-                const uint32_t buf = tile_cnt & 1;
-                ok = ptx::mbar_wait_bounded(s_full + buf, (tile_cnt >> 1) & 1, tmo);
+                const uint32_t buf = tile_cnt % NS;
+                ok = ptx::mbar_wait_bounded(s_full + buf, (tile_cnt / NS) & 1, tmo);
                 if (!ok) break;
                 ptx::tc_fence_after();
                 float x[64];

@@ -56,6 +56,7 @@ struct MainArgs {
     uint32_t* status;
     unsigned long long timeout_ns;
     int stall_unit;   // test hook: skip this TMA unit in CTA 0 (-1 = off)
+    int prefetch_tiles;  // KV tiles to prefetch into L2 ahead of the loads (0 = off)
 };
 
 template <int G>

@@ -79,14 +79,26 @@ int choose_group_rows(int R) {
     return (R % 32 == 0) ? 32 : 16;
 }
 
-// pair-kernel ring depths: K chunks (8 KB each) and V slots (32 KB each)
-constexpr int kPairNK = 5;
-constexpr int kPairNV = 3;
-using PairC = mla::PairCfg<kPairNK, kPairNV>;
+// pair-kernel ring depths: K chunks (8 KB each), V slots (32 KB each) and S
+// buffers in TMEM (PV trails S by kPairNS - 1 tiles)
+#ifndef MLA_PAIR_NK
+#define MLA_PAIR_NK 5
+#endif
+#ifndef MLA_PAIR_NV
+#define MLA_PAIR_NV 3
+#endif
+#ifndef MLA_PAIR_NS
+#define MLA_PAIR_NS 3
+#endif
+constexpr int kPairNK = MLA_PAIR_NK;
+constexpr int kPairNV = MLA_PAIR_NV;
+constexpr int kPairNS = MLA_PAIR_NS;
+constexpr int kDefaultPrefetchTiles = 2;
+using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS>;
 
 mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                        const CUtensorMap& tm_v, const mla::MainArgs& args, cudaStream_t stream) {
-    auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV>;
+    auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV, kPairNS>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairC::kSmemBytes) != cudaSuccess)
         return MLA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(2 * plan.num_partitions * plan.num_groups));
@@ -190,6 +202,7 @@ mla_status mla_decode_plan_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_ma
     if (P > 4096) P = 4096;
     p.num_partitions = P;
     p.tile_kv = mla::kTileKV;
+    p.l2_prefetch_tiles = kDefaultPrefetchTiles;
     p.workspace_bytes = workspace_layout(P, R).total;
     *plan = p;
     if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
@@ -221,6 +234,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     if (pl.B < 1 || pl.Sq < 1 || pl.H < 1 || pl.L_max < 1 || pl.num_partitions < 1 || pl.num_groups < 1 ||
         pl.group_rows * pl.num_groups != R)
         return MLA_ERR_INVALID_ARG;
+    if (pl.l2_prefetch_tiles < 0 || pl.l2_prefetch_tiles > 16) return MLA_ERR_INVALID_ARG;
     if (pl.kernel == MLA_KERNEL_TRANSPOSED) {
         if (pl.group_rows != 16 && pl.group_rows != 32) return MLA_ERR_INVALID_ARG;
     } else if (pl.kernel == MLA_KERNEL_PAIR) {
@@ -281,6 +295,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     const unsigned long long tmo = g_timeout_ns.load();
     a.timeout_ns = tmo ? tmo : kDefaultTimeoutNs;
     a.stall_unit = g_stall_unit.load();
+    a.prefetch_tiles = pl.l2_prefetch_tiles;
 
     if (phases & 1) {
         mla_status st;
