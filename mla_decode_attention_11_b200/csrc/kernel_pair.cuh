@@ -33,9 +33,15 @@
 // GEMMs split B along different axes (kv rows for S, value columns for PV),
 // so the value rows this CTA owns for S cannot double as its PV operand.
 //
-// Warp roles (224 threads): warps 0-3 softmax + epilogue (thread = TMEM lane),
+// Warp roles (256 threads): warps 0-3 softmax + epilogue (thread = TMEM lane),
 // warp 4 Q/K producer, warp 5 V producer, warp 6 TMEM allocator and (in the
-// leader CTA) the single MMA-issuing thread.  Loads of both CTAs are counted on
+// leader CTA) the QK^T issuer, warp 7 the PV issuer (leader) or the P-ready
+// forwarder (follower).  Issuing a pair MMA, checking a barrier and committing
+// each cost tens of cycles of the issuing thread, more than an N = 128 MMA
+// takes to execute, so the two GEMMs are issued from two threads.  A
+// cluster-scope release arrive costs a thread over a thousand cycles, so the
+// softmax warps only ever arrive at CTA scope: the follower's P-ready barrier
+// is forwarded to the leader by one otherwise idle thread.  Loads of both CTAs are counted on
 // the leader's barriers (2-SM TMA); MMA completion is multicast to both CTAs.
 // Every wait is bounded; on expiry a CTA records kStatusTimeout and unwinds.
 #pragma once
@@ -50,9 +56,9 @@
 
 namespace mla {
 
-template <int NK, int NV, int NS>
+template <int NK, int NV, int NS, int NP>
 struct PairCfg {
-    static constexpr int kThreads = 224;
+    static constexpr int kThreads = 256;
     static constexpr int kRows = 64;                          // query rows per CTA
     static constexpr int kQChunk = kRows * 128;               // 8 KB
     static constexpr int kKChunk = 64 * 128;                  // 8 KB (64 own kv rows)
@@ -63,11 +69,13 @@ struct PairCfg {
     static constexpr int OFF_K = OFF_Q + kNumChunks * kQChunk;
     static constexpr int OFF_V = OFF_K + NK * kKChunk;
     static constexpr int OFF_P = OFF_V + NV * kVSlot;
-    static constexpr int OFF_RED = OFF_P + 2 * kPChunk;        // floats: [2][128] max, [128] sum
+    static constexpr int kPBuf = 2 * kPChunk;                 // one P tile (2 chunks of 64 keys)
+    static_assert(NP == 1 || NP == 2, "P buffers");
+    static constexpr int OFF_RED = OFF_P + NP * kPBuf;         // floats: [2][128] max, [128] sum
     static constexpr int OFF_BAR = OFF_RED + 384 * 4;
-    // q_full, q_empty, p_full, pv_done, drain, group_sync, s_full[NS], k_full[NK], k_empty[NK],
-    // v_full[NV], v_empty[NV]
-    static constexpr int kNumBars = 6 + NS + 2 * NK + 2 * NV;
+    // q_full, q_empty, pv_done[NP], drain_s, drain_pv, group_sync, s_full[NS], p_full[NS], p_local[NS],
+    // k_full[NK], k_empty[NK], v_full[NV], v_empty[NV]
+    static constexpr int kNumBars = 6 + NP + 3 * NS + 2 * NK + 2 * NV;
     static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
     static constexpr int kSmemBytes = OFF_MISC + 64;
     static constexpr uint32_t kTmemCols = 512;                 // O: [0,256), S buffers from 256, 64 each
@@ -78,11 +86,11 @@ struct PairCfg {
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
-template <int NK, int NV, int NS>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
+template <int NK, int NV, int NS, int NP>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                            const __grid_constant__ CUtensorMap tm_v, const MainArgs args) {
-    using C = PairCfg<NK, NV, NS>;
+    using C = PairCfg<NK, NV, NS, NP>;
     extern __shared__ __align__(1024) uint8_t smem[];
 
     uint8_t* q_smem = smem + C::OFF_Q;
@@ -93,12 +101,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_full = bars + 0;
     uint64_t* q_empty = bars + 1;
-    uint64_t* p_full = bars + 2;
-    uint64_t* pv_done = bars + 3;
-    uint64_t* drain = bars + 4;
-    uint64_t* group_sync = bars + 5;
-    uint64_t* s_full = bars + 6;     // [NS]
-    uint64_t* k_full = s_full + NS;
+    uint64_t* pv_done = bars + 2;           // [NP] the PV that read P buffer b has completed
+    uint64_t* drain_s = pv_done + NP;
+    uint64_t* drain_pv = drain_s + 1;
+    uint64_t* group_sync = drain_pv + 1;
+    uint64_t* s_full = group_sync + 1;      // [NS] S buffer b holds a finished QK^T
+    uint64_t* p_full = s_full + NS;         // [NS] leader: the tile in S buffer b is through both softmaxes
+                                            //      (its S read, its P written in both CTAs)
+    uint64_t* p_local = p_full + NS;        // [NS] follower: the same, for this CTA's 128 softmax threads
+    uint64_t* k_full = p_local + NS;
     uint64_t* k_empty = k_full + NK;
     uint64_t* v_full = k_empty + NK;
     uint64_t* v_empty = v_full + NV;
@@ -123,10 +134,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     if (threadIdx.x == 0) {
         ptx::mbar_init(q_full, 1);
         ptx::mbar_init(q_empty, 1);
-        for (int i = 0; i < NS; ++i) ptx::mbar_init(s_full + i, 1);
-        ptx::mbar_init(p_full, 256);  // every softmax thread of both CTAs
-        ptx::mbar_init(pv_done, 1);
-        ptx::mbar_init(drain, 1);
+        for (int i = 0; i < NS; ++i) {
+            ptx::mbar_init(s_full + i, 1);
+            ptx::mbar_init(p_full + i, 129);   // leader's 128 softmax threads + the follower's forwarder
+            ptx::mbar_init(p_local + i, 128);  // follower's 128 softmax threads
+        }
+        for (int i = 0; i < NP; ++i) ptx::mbar_init(pv_done + i, 1);
+        ptx::mbar_init(drain_s, 1);
+        ptx::mbar_init(drain_pv, 1);
         ptx::mbar_init(group_sync, 128);
         for (int i = 0; i < NK; ++i) {
             ptx::mbar_init(k_full + i, 1);
@@ -183,7 +198,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
     }
     // shared::cluster addresses of the leader's barriers
     const uint32_t lead_q_full = ptx::mapa_shared(ptx::smem_u32(q_full), 0);
-    const uint32_t lead_p_full = ptx::mapa_shared(ptx::smem_u32(p_full), 0);
     const bool stall_cta = (blockIdx.x == 0);
 
     if (warp == 4) {
@@ -263,80 +277,119 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
         }
         __syncwarp();
     } else if (warp == 6) {
-        // ============================================================ MMA issuer (leader only)
+        // ============================================================ QK^T issuer (leader only)
         if (leader && ptx::elect_one()) {
-            uint32_t k_cnt = 0, v_cnt = 0, piece_cnt = 0, tile_cnt = 0;
             bool ok = true;
-            const uint32_t q_base = ptx::smem_u32(q_smem);
-            const uint32_t k_base = ptx::smem_u32(k_smem);
-            const uint32_t v_base = ptx::smem_u32(v_smem);
-            const uint32_t p_base = ptx::smem_u32(p_smem);
             constexpr uint16_t kBoth = 0x3;
-            // O += P . V for global tile index u
-            auto issue_pv = [&](uint32_t u, bool first_of_piece) -> bool {
-                if (!ptx::mbar_wait_bounded_cluster(p_full, u & 1, tmo)) return false;
-                ptx::tc_fence_after();
-                for (int i = 0; i < 2; ++i) {
-                    const uint32_t s = v_cnt % NV;
-                    if (!ptx::mbar_wait_bounded(v_full + s, (v_cnt / NV) & 1, tmo)) return false;
-                    ptx::tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kTileKV / 16; ++kk) {
-                        const uint64_t da = ptx::make_smem_desc(p_base + (kk >> 2) * C::kPChunk + (kk & 3) * 32, 16,
-                                                                1024, ptx::Swizzle::B128);
-                        const uint64_t db = ptx::make_smem_desc(v_base + s * C::kVSlot + kk * 2048, C::kVChunk, 1024,
-                                                                ptx::Swizzle::B128);
-                        ptx::mma_bf16_ss_pair(tmem_base + 128 * i, da, db, C::kIdescPV,
-                                              (first_of_piece && kk == 0) ? 0u : 1u);
-                    }
-                    ptx::mma_commit_pair_mc(v_empty + s, kBoth);
-                    ++v_cnt;
-                }
-                ptx::mma_commit_pair_mc(pv_done, kBoth);
-                return true;
-            };
-            // S(t) for global tile index u into S buffer u % NS
-            auto issue_s = [&](uint32_t u, bool last_of_piece) -> bool {
-                const uint32_t tm_S = tmem_base + C::kColS + 64 * (u % NS);
-                for (int jj = 0; jj < kNumChunks; ++jj) {
-                    const int j = (jj == 0) ? 8 : jj - 1;  // rope chunk first
-                    const uint32_t s = k_cnt % NK;
-                    if (!ptx::mbar_wait_bounded(k_full + s, (k_cnt / NK) & 1, tmo)) return false;
-                    ptx::tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t da = ptx::make_smem_desc(q_base + j * C::kQChunk + kk * 32, 16, 1024,
-                                                                ptx::Swizzle::B128);
-                        const uint64_t db = ptx::make_smem_desc(k_base + s * C::kKChunk + kk * 32, 16, 1024,
-                                                                ptx::Swizzle::B128);
-                        ptx::mma_bf16_ss_pair(tm_S, da, db, C::kIdescS, (jj | kk) ? 1u : 0u);
-                    }
-                    ptx::mma_commit_pair_mc(k_empty + s, kBoth);
-                    ++k_cnt;
-                }
-                if (last_of_piece) ptx::mma_commit_pair_mc(q_empty, kBoth);
-                ptx::mma_commit_pair_mc(s_full + (u % NS), kBoth);
-                return true;
-            };
-            // PV trails S by NS-1 tiles, so the softmax of a tile overlaps the
-            // QK^T of the next NS-1 tiles.
-            constexpr int kLag = NS - 1;
+            // descriptors of the chunk / slot bases; an MMA adds (byte offset >> 4)
+            const uint64_t dq0 = ptx::make_smem_desc(ptx::smem_u32(q_smem), 16, 1024, ptx::Swizzle::B128);
+            const uint64_t dk0 = ptx::make_smem_desc(ptx::smem_u32(k_smem), 16, 1024, ptx::Swizzle::B128);
+            uint32_t ks = 0, kph = 0;        // K ring slot and phase
+            uint32_t sb = 0, sph = 0;        // S buffer and its use parity
+            uint32_t u = 0, piece_cnt = 0;   // global tile index, piece count
             Piece pc;
             while (ok && walker.next(pc)) {
-                const int n = pc.tile_hi - pc.tile_lo;
                 ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
-                const uint32_t u0 = tile_cnt;  // global index of the piece's first tile
-                for (int i = 0; ok && i < n + kLag; ++i) {
-                    if (i < n) ok = issue_s(u0 + i, i == n - 1);
-                    if (ok && i >= kLag) ok = issue_pv(u0 + i - kLag, i - kLag == 0);
+                for (int t = pc.tile_lo; ok && t < pc.tile_hi; ++t) {
+                    // S buffer sb was last filled by tile u - NS: both softmaxes must be done with it
+                    if (u >= static_cast<uint32_t>(NS)) {
+                        ok = ptx::mbar_wait_bounded_cluster(p_full + sb, sph ^ 1, tmo);
+                        if (!ok) break;
+                    }
+                    const uint32_t tm_S = tmem_base + C::kColS + 64 * sb;
+                    for (int jj = 0; jj < kNumChunks; ++jj) {
+                        const uint32_t j = (jj == 0) ? 8u : static_cast<uint32_t>(jj - 1);  // rope chunk first
+                        ok = ptx::mbar_wait_bounded(k_full + ks, kph, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        const uint64_t da = dq0 + ((j * C::kQChunk) >> 4);
+                        const uint64_t db = dk0 + ((ks * C::kKChunk) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            ptx::mma_bf16_ss_pair(tm_S, da + 2 * kk, db + 2 * kk, C::kIdescS, (jj | kk) ? 1u : 0u);
+                        ptx::mma_commit_pair_mc(k_empty + ks, kBoth);
+                        if (++ks == NK) {
+                            ks = 0;
+                            kph ^= 1;
+                        }
+                    }
+                    if (!ok) break;
+                    if (t == pc.tile_hi - 1) ptx::mma_commit_pair_mc(q_empty, kBoth);
+                    ptx::mma_commit_pair_mc(s_full + sb, kBoth);
+                    if (++sb == NS) {
+                        sb = 0;
+                        sph ^= 1;
+                    }
+                    ++u;
                 }
-                tile_cnt += n;
                 ++piece_cnt;
             }
             if (!ok) atomicOr(args.status, kStatusTimeout);
-            // drain: every MMA issued must complete before TMEM is freed
-            ptx::mma_commit_pair_mc(drain, 0x1);
-            ptx::mbar_wait_bounded(drain, 0, tmo);
+            // drain: every MMA this thread issued must complete before TMEM is freed
+            ptx::mma_commit_pair_mc(drain_s, 0x1);
+            ptx::mbar_wait_bounded(drain_s, 0, tmo);
+        }
+        __syncwarp();
+    } else if (warp == 7 && !leader) {
+        // ============================================================ P-ready forwarder (follower)
+        // One cluster-scope release per tile, made here instead of by every softmax thread.
+        if (ptx::elect_one()) {
+            bool ok = true;
+            uint32_t u = 0;
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                for (int t = pc.tile_lo; ok && t < pc.tile_hi; ++t, ++u) {
+                    const uint32_t b = u % NS;
+                    ok = ptx::mbar_wait_bounded(p_local + b, (u / NS) & 1, tmo);
+                    if (ok) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(p_full + b), 0));
+                }
+            }
+            if (!ok) atomicOr(args.status, kStatusTimeout);
+        }
+        __syncwarp();
+    } else if (warp == 7) {
+        // ============================================================ PV issuer (leader only)
+        if (leader && ptx::elect_one()) {
+            bool ok = true;
+            constexpr uint16_t kBoth = 0x3;
+            const uint64_t dp0 = ptx::make_smem_desc(ptx::smem_u32(p_smem), 16, 1024, ptx::Swizzle::B128);
+            const uint64_t dv0 = ptx::make_smem_desc(ptx::smem_u32(v_smem), C::kVChunk, 1024, ptx::Swizzle::B128);
+            uint32_t vs = 0, vph = 0;  // V ring slot and phase
+            uint32_t u = 0;            // global tile index
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                for (int t = pc.tile_lo; ok && t < pc.tile_hi; ++t) {
+                    const bool first = (t == pc.tile_lo);  // O starts over for a new piece
+                    const uint32_t pb = (NP == 2) ? (u & 1) : 0;
+                    ok = ptx::mbar_wait_bounded_cluster(p_full + (u % NS), (u / NS) & 1, tmo);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    const uint64_t dpb = dp0 + ((pb * C::kPBuf) >> 4);
+                    for (int i = 0; i < 2; ++i) {
+                        ok = ptx::mbar_wait_bounded(v_full + vs, vph, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        const uint64_t db = dv0 + ((vs * C::kVSlot) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < kTileKV / 16; ++kk) {
+                            const uint64_t da = dpb + (((kk >> 2) * C::kPChunk + (kk & 3) * 32) >> 4);
+                            ptx::mma_bf16_ss_pair(tmem_base + 128 * i, da, db + ((kk * 2048) >> 4), C::kIdescPV,
+                                                  (first && kk == 0) ? 0u : 1u);
+                        }
+                        ptx::mma_commit_pair_mc(v_empty + vs, kBoth);
+                        if (++vs == NV) {
+                            vs = 0;
+                            vph ^= 1;
+                        }
+                    }
+                    if (!ok) break;
+                    ptx::mma_commit_pair_mc(pv_done + pb, kBoth);
+                    ++u;
+                }
+            }
+            if (!ok) atomicOr(args.status, kStatusTimeout);
+            ptx::mma_commit_pair_mc(drain_pv, 0x1);
+            ptx::mbar_wait_bounded(drain_pv, 0, tmo);
         }
         __syncwarp();
     } else {
@@ -369,16 +422,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
                 ptx::tc_fence_after();
                 float x[64];
                 {
-                    uint32_t rr[32];
+                    uint32_t ra[32], rb[32];
+                    ptx::tmem_ld_32(lane_addr + C::kColS + 64 * buf, ra);
+                    ptx::tmem_ld_32(lane_addr + C::kColS + 64 * buf + 32, rb);
+                    ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int c0 = 0; c0 < 64; c0 += 32) {
-                        ptx::tmem_ld_32(lane_addr + C::kColS + 64 * buf + c0, rr);
-                        ptx::tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int kv = kv0 + c0 + j;
-                            x[c0 + j] = (kv >= lo && kv < pc.L) ? __uint_as_float(rr[j]) * args.scale_log2 : -INFINITY;
-                        }
+                    for (int j = 0; j < 32; ++j) {
+                        const int kv = kv0 + j;
+                        x[j] = (kv >= lo && kv < pc.L) ? __uint_as_float(ra[j]) * args.scale_log2 : -INFINITY;
+                        const int kv2 = kv0 + 32 + j;
+                        x[32 + j] = (kv2 >= lo && kv2 < pc.L) ? __uint_as_float(rb[j]) * args.scale_log2 : -INFINITY;
                     }
                 }
                 float mloc = x[0];
@@ -389,62 +442,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(224, 1)
                 ok = group_barrier();
                 if (!ok) break;
                 const float mrow = fmaxf(mloc, redmax[L_id ^ 64]);
-                if (!first) {
-                    // P and O are free once the previous tile's PV has completed
-                    ok = ptx::mbar_wait_bounded(pv_done, (tile_cnt - 1) & 1, tmo);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                }
+                // reference max: the tile's row max on a piece's first tile, else
+                // raised lazily only when the row max grew by more than 8 (p <= 2^8)
+                float alpha = 1.f;
+                bool grow = false;
                 if (first) {
                     m_ref = mrow;
-                } else {
-                    // lazy rescale: only when the row max grew by more than 8 (p <= 2^8 otherwise)
-                    const bool grow = mrow > m_ref + 8.f;
-                    if (__any_sync(0xffffffffu, grow)) {
-                        float alpha = 1.f;
-                        if (grow) {
-                            alpha = ex2_approx(m_ref - mrow);
-                            m_ref = mrow;
-                            l_part *= alpha;
-                        }
-#pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-#pragma unroll
-                            for (int c0 = 0; c0 < 128; c0 += 32) {
-                                uint32_t rr[32];
-                                ptx::tmem_ld_32(lane_addr + 128 * i + c0, rr);
-                                ptx::tmem_wait_ld();
-#pragma unroll
-                                for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * alpha);
-                                ptx::tmem_st_32(lane_addr + 128 * i + c0, rr);
-                            }
-                        }
-                        ptx::tmem_wait_st();
-                    }
+                } else if (mrow > m_ref + 8.f) {
+                    grow = true;
+                    alpha = ex2_approx(m_ref - mrow);
+                    m_ref = mrow;
+                    l_part *= alpha;
                 }
-                // P[r][64h .. 64h+63] = exp2(x - m_ref) as bf16, K-major 128-byte swizzled
-                uint8_t* prow = p_smem + h * C::kPChunk + r * 128;
+                const bool warp_grow = __any_sync(0xffffffffu, grow);
+                // P[r][64h .. 64h+63] = exp2(x - m_ref) as bf16, computed before waiting
+                uint32_t packed[32];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float a0 = ex2_approx(x[8 * u + 2 * e] - m_ref);
-                        const float a1 = ex2_approx(x[8 * u + 2 * e + 1] - m_ref);
-                        l_part += a0 + a1;
-                        const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
-                        w4[e] = *reinterpret_cast<const uint32_t*>(&hv);
-                    }
-                    *reinterpret_cast<uint4*>(prow + ((u ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                for (int e = 0; e < 32; ++e) {
+                    const float a0 = ex2_approx(x[2 * e] - m_ref);
+                    const float a1 = ex2_approx(x[2 * e + 1] - m_ref);
+                    l_part += a0 + a1;
+                    const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+                    packed[e] = *reinterpret_cast<const uint32_t*>(&hv);
                 }
+                const uint32_t pb = (NP == 2) ? (tile_cnt & 1) : 0;
+                // the P buffer is free once the PV that last read it completed
+                // (NP = 1: the previous tile's; NP = 2: the one two tiles back)
+                if (NP == 1 ? !first : (t >= pc.tile_lo + 2)) {
+                    const uint32_t v = tile_cnt - NP;
+                    ok = ptx::mbar_wait_bounded(pv_done + pb, (NP == 2) ? ((v >> 1) & 1) : (v & 1), tmo);
+                    if (!ok) break;
+                }
+                if (warp_grow) {
+                    // O must hold every earlier tile before it is rescaled
+                    if (NP == 2) {
+                        const uint32_t v = tile_cnt - 1;
+                        ok = ptx::mbar_wait_bounded(pv_done + (v & 1), (v >> 1) & 1, tmo);
+                        if (!ok) break;
+                    }
+                    ptx::tc_fence_after();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+#pragma unroll
+                        for (int c0 = 0; c0 < 128; c0 += 32) {
+                            uint32_t rr[32];
+                            ptx::tmem_ld_32(lane_addr + 128 * i + c0, rr);
+                            ptx::tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) rr[j] = __float_as_uint(__uint_as_float(rr[j]) * alpha);
+                            ptx::tmem_st_32(lane_addr + 128 * i + c0, rr);
+                        }
+                    }
+                    ptx::tmem_wait_st();
+                }
+                uint8_t* prow = p_smem + pb * C::kPBuf + h * C::kPChunk + r * 128;
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu)
+                    *reinterpret_cast<uint4*>(prow + ((uu ^ (r & 7)) << 4)) =
+                        make_uint4(packed[4 * uu + 0], packed[4 * uu + 1], packed[4 * uu + 2], packed[4 * uu + 3]);
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive_cluster(lead_p_full);
+                // CTA-scope arrive: the leader's own barrier, or the follower's local one
+                ptx::mbar_arrive(leader ? (p_full + buf) : (p_local + buf));
                 ++tile_cnt;
             }
             if (!ok) break;
             // ---------------- epilogue: O / l -> out (or a partial), lse
-            ok = ptx::mbar_wait_bounded(pv_done, (tile_cnt - 1) & 1, tmo);
+            {
+                const uint32_t v = tile_cnt - 1;  // the piece's last tile
+                ok = (NP == 2) ? ptx::mbar_wait_bounded(pv_done + (v & 1), (v >> 1) & 1, tmo)
+                               : ptx::mbar_wait_bounded(pv_done, v & 1, tmo);
+            }
             if (!ok) break;
             ptx::tc_fence_after();
             float* redsum = red + 256;

@@ -82,23 +82,27 @@ int choose_group_rows(int R) {
 // pair-kernel ring depths: K chunks (8 KB each), V slots (32 KB each) and S
 // buffers in TMEM (PV trails S by kPairNS - 1 tiles)
 #ifndef MLA_PAIR_NK
-#define MLA_PAIR_NK 5
+#define MLA_PAIR_NK 7
 #endif
 #ifndef MLA_PAIR_NV
-#define MLA_PAIR_NV 3
+#define MLA_PAIR_NV 2
 #endif
 #ifndef MLA_PAIR_NS
 #define MLA_PAIR_NS 3
 #endif
+#ifndef MLA_PAIR_NP
+#define MLA_PAIR_NP 2
+#endif
 constexpr int kPairNK = MLA_PAIR_NK;
 constexpr int kPairNV = MLA_PAIR_NV;
 constexpr int kPairNS = MLA_PAIR_NS;
+constexpr int kPairNP = MLA_PAIR_NP;  // P buffers in shared memory
 constexpr int kDefaultPrefetchTiles = 2;
-using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS>;
+using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS, kPairNP>;
 
 mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                        const CUtensorMap& tm_v, const mla::MainArgs& args, cudaStream_t stream) {
-    auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV, kPairNS>;
+    auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV, kPairNS, kPairNP>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairC::kSmemBytes) != cudaSuccess)
         return MLA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(2 * plan.num_partitions * plan.num_groups));
