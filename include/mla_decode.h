@@ -177,6 +177,47 @@ mla_status mla_decode_run_phase(const mla_plan* plan, const void* q, const void*
  */
 mla_status mla_decode_check(const mla_plan* plan, void* workspace, void* stream);
 
+/*
+ * mla_decode_run_noalloc -- mla_decode_run without a caller workspace.  The
+ * decode papers have no counterpart to this call; it exists for callers that
+ * must not allocate device memory while decoding: a serving engine that hands
+ * almost all HBM to its KV cache at start-up and cannot spare a workspace
+ * later, or a plain C host that has no device allocator to draw from.
+ *
+ * The split-KV partials and the status words live in one static device array
+ * of MLA_NOALLOC_SCRATCH_BYTES inside this library.  Every GPU that loads the
+ * library holds that array until the process exits; the call itself allocates
+ * nothing (no cudaMalloc, no cudaFree, no allocating library routine).
+ *
+ *   plan, q, kv, seqlens, softmax_scale, out, lse, stream
+ *             as for mla_decode_run; inputs and outputs are still the
+ *             caller's device buffers
+ *   wait_and_check
+ *             0: only enqueue, like mla_decode_run; device-recorded faults are
+ *             then not reported (the next call clears them).
+ *             non-zero: also synchronize `stream` and read the status words,
+ *             returning MLA_ERR_TIMEOUT or MLA_ERR_SEQLEN like mla_decode_check
+ *
+ * The first call on a device looks up the array's device address there (with
+ * that device current), which may load the library's device code onto it:
+ * make that first call outside any stream capture.  Each call clears the
+ * status words on `stream` before its launches; the partial slots keep the
+ * previous call's contents, which nothing reads.  All calls on a device share
+ * the one array, so two calls whose work can overlap on the GPU (different
+ * streams without ordering, several host threads) race and give wrong
+ * results: order them on one stream.
+ *
+ * Returns the codes of mla_decode_run, plus MLA_ERR_WORKSPACE when the plan
+ * needs more than MLA_NOALLOC_SCRATCH_BYTES of scratch (every automatic plan
+ * for a 148-SM device fits; a large num_partitions_override may not), checked
+ * before anything is enqueued, and MLA_ERR_UNSUPPORTED for a device ordinal
+ * of 64 or more.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (40u * 1024u * 1024u)
+mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                                  float softmax_scale, void* out, float* lse, int32_t wait_and_check,
+                                  void* stream);
+
 /* Static English description of a status code (never NULL). */
 const char* mla_status_string(mla_status status);
 

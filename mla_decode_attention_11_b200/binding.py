@@ -7,7 +7,8 @@ device is not an sm_100 GPU, the calls raise.
 
 Entry points mirror include/mla_decode.h:
     mla_decode_plan, mla_decode_workspace_init, mla_decode_run,
-    mla_decode_check, mla_status_string, mla_decode_set_debug
+    mla_decode_check, mla_status_string, mla_decode_set_debug,
+    mla_decode_run_noalloc
 plus the convenience wrappers ``mla_decode`` (device tensors in, device
 tensors out) and ``mla_decode_host`` (host tensors in and out, with the
 copies done here around the library call).
@@ -31,9 +32,10 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_ALIGNMENT", 3
                 4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_WORKSPACE", 7: "MLA_ERR_SEQLEN"}
 MLA_KERNEL_TRANSPOSED = 1
 MLA_KERNEL_PAIR = 2
+MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
 EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
-                    "mla_decode_check",
+                    "mla_decode_check", "mla_decode_run_noalloc",
                     "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug")
 
 
@@ -91,6 +93,9 @@ def load_library(build_if_missing: bool = True):
         lib.mla_decode_run_phase.restype = c_i32
         lib.mla_decode_run_phase.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp,
                                              c_sz, c_vp, c_i32]
+        lib.mla_decode_run_noalloc.restype = c_i32
+        lib.mla_decode_run_noalloc.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_i32,
+                                               c_vp]
         lib.mla_decode_check.restype = c_i32
         lib.mla_decode_check.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp]
         lib.mla_status_string.restype = ctypes.c_char_p
@@ -187,6 +192,33 @@ def mla_decode_run_phase(plan: mla_plan, q: torch.Tensor, kv: torch.Tensor, seql
                                              int(phase))
     if rc != MLA_OK:
         raise MlaError(rc, "mla_decode_run_phase")
+
+
+def mla_decode_run_noalloc(plan: mla_plan, q: torch.Tensor, kv: torch.Tensor, seqlens: torch.Tensor,
+                           softmax_scale: float, out: torch.Tensor, lse: torch.Tensor, wait_and_check: bool = False,
+                           stream=None) -> None:
+    """mla_decode_run for callers that may not allocate device memory while
+    decoding (an engine whose KV cache took nearly all HBM at start-up, a C host
+    without a device allocator): the library's own static scratch array of
+    MLA_NOALLOC_SCRATCH_BYTES per device stands in for the workspace.  Calls on
+    one device share that array, so calls that may overlap on the GPU race;
+    make the first call on a device outside stream capture.  With
+    wait_and_check the stream is synchronised and a recorded device fault
+    raises, as mla_decode_check does."""
+    B, Sq, H, L = plan.B, plan.Sq, plan.H, plan.L_max
+    _check_tensor(q, "q", torch.bfloat16, (B, Sq, H, D_QK))
+    _check_tensor(kv, "kv", torch.bfloat16, (B, L, D_QK))
+    _check_tensor(seqlens, "seqlens", torch.int32, (B,))
+    _check_tensor(out, "out", torch.bfloat16, (B, Sq, H, D_V))
+    _check_tensor(lse, "lse", torch.float32, (B, Sq, H))
+    rc = load_library().mla_decode_run_noalloc(ctypes.byref(plan), q.data_ptr(), kv.data_ptr(), seqlens.data_ptr(),
+                                               float(softmax_scale), out.data_ptr(), lse.data_ptr(),
+                                               int(bool(wait_and_check)), _stream_handle(stream))
+    if rc != MLA_OK:
+        what = "mla_decode_run_noalloc"
+        if rc == 6:
+            what += f" (plan needs more than the {MLA_NOALLOC_SCRATCH_BYTES} bytes of static scratch)"
+        raise MlaError(rc, what)
 
 
 def mla_decode_check(plan: mla_plan, workspace: torch.Tensor, stream=None) -> int:

@@ -372,3 +372,84 @@ mla_status mla_decode_set_debug(uint64_t wait_timeout_ns, int32_t stall_tile) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Run variant that allocates nothing: its split-KV partials and status words
+// live in one file-scope device array instead of a caller workspace.  It is
+// for callers that may not allocate device memory on the decode path, e.g. a
+// serving engine that reserved nearly all HBM for its KV cache at start-up, or
+// a C host with no device allocator of its own.  Every GPU that loads this
+// library holds the array (MLA_NOALLOC_SCRATCH_BYTES) until the process exits.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device `dev`.  The name
+// g_noalloc_scratch is only a host-side handle; the address comes from
+// cudaGetSymbolAddress, taken once per device while that device is current.
+mla_status noalloc_scratch(int dev, void** ptr) {
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return MLA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return MLA_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                                  float softmax_scale, void* out, float* lse, int32_t wait_and_check,
+                                  void* stream_) {
+    if (!plan) return MLA_ERR_INVALID_ARG;
+    if (plan->num_partitions < 1 || plan->num_partitions > 4096 || plan->Sq < 1 || plan->H < 1)
+        return MLA_ERR_INVALID_ARG;
+    const size_t need = workspace_layout(plan->num_partitions, plan->Sq * plan->H).total;
+    if (need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    void* scratch = nullptr;
+    mla_status st = noalloc_scratch(dev, &scratch);
+    if (st != MLA_OK) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    // the status words must start at zero; the partial slots are always
+    // written before they are read, so what an earlier call left there is
+    // harmless
+    if (cudaMemsetAsync(scratch, 0, kHeaderBytes, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    st = run_phases(plan, q, kv, seqlens, softmax_scale, out, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream_, 3);
+    if (st != MLA_OK || !wait_and_check) return st;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, scratch, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (word & mla::kStatusTimeout) return MLA_ERR_TIMEOUT;
+    if (word & mla::kStatusSeqlen) return MLA_ERR_SEQLEN;
+    return MLA_OK;
+}
+
+}  // extern "C"
