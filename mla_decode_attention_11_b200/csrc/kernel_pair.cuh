@@ -206,6 +206,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             uint32_t k_cnt = 0, piece_cnt = 0;
             int unit = 0;
             bool ok = true;
+            // L2 prefetch cursor, `prefetch_tiles` tiles ahead of the K loads
+            // through this partition's tiles, across piece boundaries.  A tile
+            // is prefetched whole (all 128 rows, K and V columns alike); on
+            // entering a later piece the cursor also prefetches that piece's
+            // Q rows, so the Q reload after a piece boundary hits L2.  The two
+            // CTAs split the column chunks.
+            PieceWalker pf_walker = walker;
+            Piece pf_pc;
+            bool pf_live = args.prefetch_tiles > 0 && pf_walker.next(pf_pc);
+            int pf_t = pf_live ? pf_pc.tile_lo : 0;
+            auto prefetch_next = [&]() {
+                if (!pf_live) return;
+                int row0 = pf_t * kTileKV;
+                if (row0 + kTileKV > pf_pc.L) row0 = pf_pc.L - kTileKV;
+                for (int j = static_cast<int>(rank); j < kNumChunks; j += 2)
+                    ptx::tma_prefetch_3d(&tm_v, j * kChunk, row0, pf_pc.b);
+                if (++pf_t == pf_pc.tile_hi) {
+                    pf_live = pf_walker.next(pf_pc);
+                    if (pf_live) {
+                        pf_t = pf_pc.tile_lo;
+                        const int qrow = pf_pc.b * args.R + g * 128 + static_cast<int>(rank) * 64;
+                        for (int c = 0; c < kNumChunks; ++c) ptx::tma_prefetch_2d(&tm_q, c * kChunk, qrow);
+                    }
+                }
+            };
+            for (int i = 0; i < args.prefetch_tiles; ++i) prefetch_next();
             Piece pc;
             while (ok && walker.next(pc)) {
                 if (piece_cnt > 0) ok = ptx::mbar_wait_bounded(q_empty, (piece_cnt - 1) & 1, tmo);
@@ -217,6 +243,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                         ptx::tma_load_2d_pair(q_smem + c * C::kQChunk, &tm_q, lead_q_full, c * kChunk, qrow);
                 ++unit;
                 for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    prefetch_next();
                     int row0 = t * kTileKV;
                     if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
                     const int krow = row0 + static_cast<int>(rank) * 64;
@@ -244,19 +271,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         if (ptx::elect_one()) {
             uint32_t v_cnt = 0;
             bool ok = true;
-            const int pf = args.prefetch_tiles;
-            // L2 prefetch of a whole tile, split between the two CTAs by column chunk
-            auto prefetch_tile = [&](const Piece& pc, int t) {
-                int row0 = t * kTileKV;
-                if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
-                for (int j = static_cast<int>(rank); j < kNumChunks; j += 2)
-                    ptx::tma_prefetch_3d(&tm_v, j * kChunk, row0, pc.b);
-            };
             Piece pc;
             while (ok && walker.next(pc)) {
-                for (int t = pc.tile_lo; t < pc.tile_lo + pf && t < pc.tile_hi; ++t) prefetch_tile(pc, t);
                 for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
-                    if (pf > 0 && t + pf < pc.tile_hi) prefetch_tile(pc, t + pf);
                     int row0 = t * kTileKV;
                     if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
                     for (int i = 0; i < 2; ++i) {

@@ -97,7 +97,7 @@ constexpr int kPairNK = MLA_PAIR_NK;
 constexpr int kPairNV = MLA_PAIR_NV;
 constexpr int kPairNS = MLA_PAIR_NS;
 constexpr int kPairNP = MLA_PAIR_NP;  // P buffers in shared memory
-constexpr int kDefaultPrefetchTiles = 2;
+constexpr int kDefaultPrefetchTiles = 1;
 using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS, kPairNP>;
 
 mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
