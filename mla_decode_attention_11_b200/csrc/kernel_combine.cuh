@@ -29,8 +29,11 @@ struct CombineArgs {
     const float* part_lse;
 };
 
-constexpr int kCombineThreads = 128;
-constexpr int kCombineRowsPerCta = 16;
+// One warp per query row, 8 rows per CTA.  The kernel is bound by the bytes of
+// the partials it reads, so each lane keeps up to 4 partials x 4 float4 in
+// flight instead of walking the partials one after another.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineRowsPerCta = kCombineThreads / 32;
 
 __global__ void __launch_bounds__(kCombineThreads)
     mla_decode_combine_kernel(const CombineArgs args) {
@@ -61,17 +64,16 @@ __global__ void __launch_bounds__(kCombineThreads)
         acc += red_acc[w];
         tot += red_tot[w];
     }
+    const int r = blockIdx.y * kCombineRowsPerCta + warp;  // this warp's query row
+    if (r >= args.R) return;
+    const size_t orow = static_cast<size_t>(b) * args.R + r;
     const int L = clamp_len(args.seqlens[b], args.L_max, nullptr);
     const long long n = num_tiles(L);
-    const int row_lo = blockIdx.y * kCombineRowsPerCta;
-    const int row_hi = min(args.R, row_lo + kCombineRowsPerCta);
-
     if (n == 0) {
-        for (int r = row_lo + warp; r < row_hi; r += kCombineThreads / 32) {
-            const size_t orow = static_cast<size_t>(b) * args.R + r;
-            for (int e = lane; e < kDv; e += 32) args.out[orow * kDv + e] = __float2bfloat16_rn(0.f);
-            if (lane == 0) args.lse[orow] = -INFINITY;
-        }
+        uint4* dst = reinterpret_cast<uint4*>(args.out + orow * kDv);  // 64 x 16 bytes
+        dst[lane] = make_uint4(0u, 0u, 0u, 0u);
+        dst[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
+        if (lane == 0) args.lse[orow] = -INFINITY;
         return;
     }
     const long long T = (tot + args.P - 1) / args.P;
@@ -79,48 +81,65 @@ __global__ void __launch_bounds__(kCombineThreads)
     const int p1 = static_cast<int>((acc + n - 1) / T);
     if (p0 == p1) return;  // finished by the main kernel
     const int k = p1 - p0 + 1;
+    // slot of the i-th piece: the first partition's piece continues after it
+    // (2 p0 + 1), every later piece started before its partition (2 p)
+    auto slot_of = [&](int i) { return (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i); };
 
-    for (int r = row_lo + warp; r < row_hi; r += kCombineThreads / 32) {
-        // pass 1: merged lse
-        float m = -INFINITY;
-        for (int i = 0; i < k; ++i) {
-            const int slot = (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i);
-            m = fmaxf(m, args.part_lse[static_cast<size_t>(slot) * args.R + r]);
-        }
-        float s = 0.f;
-        for (int i = 0; i < k; ++i) {
-            const int slot = (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i);
-            s += expf(args.part_lse[static_cast<size_t>(slot) * args.R + r] - m);
-        }
-        const float lse_all = m + logf(s);
-        // pass 2: weighted sum, 16 columns per lane (4 x float4)
-        float acc_o[16];
+    // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
+    float m = -INFINITY;
+    for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc_o[e] = 0.f;
-        for (int i = 0; i < k; ++i) {
-            const int slot = (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i);
-            const size_t prow = static_cast<size_t>(slot) * args.R + r;
-            const float w = expf(args.part_lse[prow] - lse_all);
-            const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * kDv);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+    for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const float4 x = src[v * 32 + lane];
-                acc_o[4 * v + 0] += w * x.x;
-                acc_o[4 * v + 1] += w * x.y;
-                acc_o[4 * v + 2] += w * x.z;
-                acc_o[4 * v + 3] += w * x.w;
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float lse_all = m + logf(sum);
+
+    // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
+    float4 acc_o[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < k; i0 += 4) {
+        float4 x[4][4];
+        float w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j;
+            w[j] = 0.f;
+            if (i < k) {
+                const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
+                w[j] = expf(args.part_lse[prow] - lse_all);
+                const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * kDv);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
             }
         }
-        const size_t orow = static_cast<size_t>(b) * args.R + r;
-        __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(args.out + orow * kDv);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-            const int e0 = (v * 32 + lane) * 4;  // column of acc_o[4v]
-            dst[e0 / 2] = __floats2bfloat162_rn(acc_o[4 * v + 0], acc_o[4 * v + 1]);
-            dst[e0 / 2 + 1] = __floats2bfloat162_rn(acc_o[4 * v + 2], acc_o[4 * v + 3]);
+        for (int j = 0; j < 4; ++j) {
+            if (i0 + j < k) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    acc_o[v].x += w[j] * x[j][v].x;
+                    acc_o[v].y += w[j] * x[j][v].y;
+                    acc_o[v].z += w[j] * x[j][v].z;
+                    acc_o[v].w += w[j] * x[j][v].w;
+                }
+            }
         }
-        if (lane == 0) args.lse[orow] = lse_all;
     }
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(args.out + orow * kDv);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+        const int e0 = (lane + 32 * v) * 4;  // first column of acc_o[v]
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc_o[v].x, acc_o[v].y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc_o[v].z, acc_o[v].w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(dst + e0 / 2) = pk;
+    }
+    if (lane == 0) args.lse[orow] = lse_all;
 }
 
 }  // namespace mla

@@ -210,7 +210,13 @@ def test_bounded_wait_timeout_reports_and_recovers(cuda_device, H):
         assert e.value.code == 5
     finally:
         M.mla_decode_set_debug(0, -1)
-    check_workload(w)  # the next run is clean
+    # the next run on the same workspace is clean: the check cleared the
+    # status words the abandoned run left behind
+    M.mla_decode_run(plan, q.to(dev), kv.to(dev), sl.to(dev), w.scale, out, lse, ws)
+    M.mla_decode_check(plan, ws)
+    ro, rl = oracle.mla_decode(q, kv, sl, w.scale)
+    assert_parity(out.cpu(), lse.cpu(), ro, rl, f"after timeout H{H}")
+    check_workload(w)
 
 
 # ---- full sizes, in the launch configuration bench.py times: sampled rows
