@@ -70,7 +70,7 @@ struct PairCfg {
     static constexpr int OFF_V = OFF_K + NK * kKChunk;
     static constexpr int OFF_P = OFF_V + NV * kVSlot;
     static constexpr int kPBuf = 2 * kPChunk;                 // one P tile (2 chunks of 64 keys)
-    static_assert(NP == 1 || NP == 2, "P buffers");
+    static_assert(NP == 2, "two P buffers (they double as the 32 KB epilogue stage)");
     static constexpr int OFF_RED = OFF_P + NP * kPBuf;         // floats: [2][128] max, [128] sum
     static constexpr int OFF_BAR = OFF_RED + 384 * 4;
     // q_full, q_empty, pv_done[NP], drain_s, drain_pv, group_sync, s_full[NS], p_full[NS], p_local[NS],
@@ -539,36 +539,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             const float l_row = l_part + redsum[L_id ^ 64];
             const float inv_l = 1.f / l_row;
             const int qrow = g * 128 + static_cast<int>(rank) * 64 + r;  // row within the sequence
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-#pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    uint32_t rr[32];
-                    ptx::tmem_ld_32(lane_addr + 128 * i + c0, rr);
+            // O / l leaves TMEM 64 columns at a time and is transposed through a
+            // warp-private 32 x 64 fp32 stage, so that each store instruction
+            // writes whole row segments (a thread holds one row, and direct
+            // stores would put 32 rows in every instruction).  The stage is the
+            // P buffers: every PV of the piece has completed, and the next
+            // piece's P is written only after the closing group barrier.
+            {
+                float4* stage = reinterpret_cast<float4*>(p_smem) + warp * (32 * 16);
+                const int row_base = g * 128 + static_cast<int>(rank) * 64 + 32 * (warp & 1);  // lane 0's row
+                const bool partial = (pc.slot >= 0);
+                const size_t grow0 =
+                    partial ? static_cast<size_t>(pc.slot) * args.R + row_base : static_cast<size_t>(pc.b) * args.R + row_base;
+#pragma unroll 1
+                for (int blk = 0; blk < 4; ++blk) {
+                    const int i = blk >> 1, c0 = (blk & 1) * 64;
+                    uint32_t ra[32], rb[32];
+                    ptx::tmem_ld_32(lane_addr + 128 * i + c0, ra);
+                    ptx::tmem_ld_32(lane_addr + 128 * i + c0 + 32, rb);
                     ptx::tmem_wait_ld();
-                    const int dv0 = 256 * i + 128 * h + c0;
-                    if (pc.slot < 0) {
-                        __nv_bfloat16* dst = args.out + (static_cast<size_t>(pc.b) * args.R + qrow) * kDv + dv0;
+                    float4* srow = stage + lane * 16;
 #pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            uint32_t w4[4];
+                    for (int k = 0; k < 8; ++k) {
+                        srow[k ^ (lane & 15)] =
+                            make_float4(__uint_as_float(ra[4 * k + 0]) * inv_l, __uint_as_float(ra[4 * k + 1]) * inv_l,
+                                        __uint_as_float(ra[4 * k + 2]) * inv_l, __uint_as_float(ra[4 * k + 3]) * inv_l);
+                        srow[(k + 8) ^ (lane & 15)] =
+                            make_float4(__uint_as_float(rb[4 * k + 0]) * inv_l, __uint_as_float(rb[4 * k + 1]) * inv_l,
+                                        __uint_as_float(rb[4 * k + 2]) * inv_l, __uint_as_float(rb[4 * k + 3]) * inv_l);
+                    }
+                    __syncwarp();
+                    const int col = 256 * i + 128 * h + c0;  // first value column of the block
+                    if (partial) {
+                        // 16 lanes per row: 2 rows x 256 B per instruction
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __nv_bfloat162 hv =
-                                    __floats2bfloat162_rn(__uint_as_float(rr[8 * v + 2 * e]) * inv_l,
-                                                          __uint_as_float(rr[8 * v + 2 * e + 1]) * inv_l);
-                                w4[e] = *reinterpret_cast<const uint32_t*>(&hv);
-                            }
-                            *reinterpret_cast<uint4*>(dst + 8 * v) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                        for (int it = 0; it < 16; ++it) {
+                            const int rr = 2 * it + (lane >> 4), k = lane & 15;
+                            const float4 x = stage[rr * 16 + (k ^ (rr & 15))];
+                            *reinterpret_cast<float4*>(args.part_o + (grow0 + rr) * kDv + col + 4 * k) = x;
                         }
                     } else {
-                        float* dst = args.part_o + (static_cast<size_t>(pc.slot) * args.R + qrow) * kDv + dv0;
+                        // 8 lanes per row, 8 columns each: 4 rows x 128 B of bf16 per instruction
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            *reinterpret_cast<float4*>(dst + 4 * v) =
-                                make_float4(__uint_as_float(rr[4 * v + 0]) * inv_l, __uint_as_float(rr[4 * v + 1]) * inv_l,
-                                            __uint_as_float(rr[4 * v + 2]) * inv_l, __uint_as_float(rr[4 * v + 3]) * inv_l);
+                        for (int it = 0; it < 8; ++it) {
+                            const int rr = 4 * it + (lane >> 3), k = lane & 7;
+                            const float4 x0 = stage[rr * 16 + ((2 * k) ^ (rr & 15))];
+                            const float4 x1 = stage[rr * 16 + ((2 * k + 1) ^ (rr & 15))];
+                            const __nv_bfloat162 b0 = __floats2bfloat162_rn(x0.x, x0.y);
+                            const __nv_bfloat162 b1 = __floats2bfloat162_rn(x0.z, x0.w);
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x1.x, x1.y);
+                            const __nv_bfloat162 b3 = __floats2bfloat162_rn(x1.z, x1.w);
+                            *reinterpret_cast<uint4*>(args.out + (grow0 + rr) * kDv + col + 8 * k) =
+                                make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
+                                           *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
+                        }
                     }
+                    __syncwarp();  // the stage is rewritten by the next block
                 }
             }
             if (h == 0) {
