@@ -197,14 +197,29 @@ def run_ours(args, w: W.Workload):
     M.mla_decode_workspace_init(plan, ws)
     out = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)
 
     def step():
         M.mla_decode_run(plan, qd, kvd, sld, w.scale, out, lse, ws, stream=stream)
 
-    for _ in range(args.warmup):
-        step()
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
     M.mla_decode_check(plan, ws, stream=stream)
+
+    # The K timed decodes are launched as one CUDA graph (captured, not run,
+    # here), so that the host-side cost of a call (~25 us through Python)
+    # does not leave the GPU idle between the launches of small workloads.
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    fn()
+        return g
+
+    g_steps = capture(step, args.steps)
+    torch.cuda.synchronize(dev)
 
     # ---- timed region: K full steps
     clocks = ClockSampler(local)
@@ -214,10 +229,10 @@ def run_ours(args, w: W.Workload):
     clocks.start()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
+    with torch.cuda.stream(stream):  # a graph replays on the current stream
+        e0.record(stream)
+        g_steps.replay()
+        e1.record(stream)
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
     if dist:
@@ -229,20 +244,25 @@ def run_ours(args, w: W.Workload):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         t_ms = float(t.item())
 
-    # ---- per-kernel breakdown (same work: phase 1 = main kernel, phase 2 = combine)
-    main_ms, comb_ms = [], []
-    for _ in range(max(3, min(args.steps, 50))):
-        a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        a.record(stream)
-        M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, 1, stream=stream)
-        b.record(stream)
-        M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, 2, stream=stream)
-        c.record(stream)
+    # ---- per-kernel breakdown: the same launches, each kernel alone, back to
+    # back in a graph (phase 1 = main kernel, phase 2 = split-KV combine)
+    n_brk = max(3, min(args.steps, 50))
+
+    def timed_graph(phase):
+        g = capture(lambda: M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, phase, stream=stream),
+                    n_brk)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
         torch.cuda.synchronize(dev)
-        main_ms.append(a.elapsed_time(b))
-        comb_ms.append(b.elapsed_time(c))
-    main_avg = statistics.mean(main_ms)
-    comb_avg = statistics.mean(comb_ms)
+        return a.elapsed_time(b) / n_brk
+
+    main_avg = timed_graph(1)
+    comb_avg = timed_graph(2)
+    del g_steps
+    M.mla_decode_check(plan, ws, stream=stream)
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, min(args.steps, 5))
@@ -250,16 +270,17 @@ def run_ours(args, w: W.Workload):
     outh = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16).pin_memory()
     lseh = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32).pin_memory()
     bufs = {}
-    M.mla_decode_host(qh, kvh, slh, w.scale, plan, ws, dev_bufs=bufs, out_host=outh, lse_host=lseh)
-    torch.cuda.synchronize(dev)
-    if dist:
-        dist.barrier()
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for _ in range(e2e_steps):
+    with torch.cuda.stream(stream):  # copies and launches on the bench stream
         M.mla_decode_host(qh, kvh, slh, w.scale, plan, ws, dev_bufs=bufs, out_host=outh, lse_host=lseh)
-    f1.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            M.mla_decode_host(qh, kvh, slh, w.scale, plan, ws, dev_bufs=bufs, out_host=outh, lse_host=lseh)
+        f1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = f0.elapsed_time(f1) / e2e_steps
     if dist:
