@@ -56,6 +56,12 @@ def _load():
             lib.oracle_mla_decode_rows.restype = ctypes.c_int
             lib.oracle_mla_decode_rows.argtypes = [ptr, ptr, ptr, i64, i64, i64, i64, i64, i64,
                                                    dbl, ptr, i64, ptr, ptr, ctypes.c_int]
+            lib.oracle_mla_decode_sinks.restype = ctypes.c_int
+            lib.oracle_mla_decode_sinks.argtypes = [ptr, ptr, ptr, i64, i64, i64, i64, i64, i64,
+                                                    dbl, ptr, ptr, ptr, ctypes.c_int]
+            lib.oracle_mla_decode_rows_sinks.restype = ctypes.c_int
+            lib.oracle_mla_decode_rows_sinks.argtypes = [ptr, ptr, ptr, i64, i64, i64, i64, i64, i64,
+                                                         dbl, ptr, ptr, i64, ptr, ptr, ctypes.c_int]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -78,9 +84,20 @@ def max_threads() -> int:
     return int(_load().oracle_max_threads())
 
 
-def mla_decode(q, kv, seqlens, scale: float, d_v: int = 512, num_threads: int = 0):
+def _sinks_arg(sinks, H):
+    """None -> (None, NULL); else a C-contiguous float64 [H] array and its address."""
+    if sinks is None:
+        return None, None
+    a = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(-1))
+    if a.shape[0] != H:
+        raise ValueError("sinks must have H entries")
+    return a, a.ctypes.data
+
+
+def mla_decode(q, kv, seqlens, scale: float, d_v: int = 512, num_threads: int = 0, sinks=None):
     """Oracle for every row.  q [B,Sq,H,d_qk] bf16, kv [B,L_max,d_qk] bf16,
-    seqlens int [B].  Returns (out float64 [B,Sq,H,d_v], lse float64 [B,Sq,H])."""
+    seqlens int [B], sinks None or [H] sink logits (one extra, value-free
+    softmax term per head).  Returns (out float64 [B,Sq,H,d_v], lse float64 [B,Sq,H])."""
     qb = _as_bf16_bits(q)
     kvb = _as_bf16_bits(kv)
     if qb.ndim != 4 or kvb.ndim != 3:
@@ -94,17 +111,18 @@ def mla_decode(q, kv, seqlens, scale: float, d_v: int = 512, num_threads: int = 
         raise ValueError("seqlens must have B entries")
     out = np.empty((B, Sq, H, d_v), dtype=np.float64)
     lse = np.empty((B, Sq, H), dtype=np.float64)
-    rc = _load().oracle_mla_decode(qb.ctypes.data, kvb.ctypes.data, sl.ctypes.data,
-                                   B, Sq, H, L_max, d_qk, d_v, float(scale),
-                                   out.ctypes.data, lse.ctypes.data, int(num_threads))
+    keep, sp = _sinks_arg(sinks, H)
+    rc = _load().oracle_mla_decode_sinks(qb.ctypes.data, kvb.ctypes.data, sl.ctypes.data,
+                                         B, Sq, H, L_max, d_qk, d_v, float(scale), sp,
+                                         out.ctypes.data, lse.ctypes.data, int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle_mla_decode failed with code {rc}")
     return out, lse
 
 
-def mla_decode_rows(q, kv, seqlens, scale: float, row_ids, d_v: int = 512, num_threads: int = 0):
-    """Oracle for selected flattened rows r = (b*Sq + t)*H + h.
-    Returns (out float64 [n, d_v], lse float64 [n])."""
+def mla_decode_rows(q, kv, seqlens, scale: float, row_ids, d_v: int = 512, num_threads: int = 0, sinks=None):
+    """Oracle for selected flattened rows r = (b*Sq + t)*H + h (sinks as in
+    mla_decode).  Returns (out float64 [n, d_v], lse float64 [n])."""
     qb = _as_bf16_bits(q)
     kvb = _as_bf16_bits(kv)
     B, Sq, H, d_qk = qb.shape
@@ -113,10 +131,11 @@ def mla_decode_rows(q, kv, seqlens, scale: float, row_ids, d_v: int = 512, num_t
     rows = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64).reshape(-1))
     out = np.empty((rows.shape[0], d_v), dtype=np.float64)
     lse = np.empty((rows.shape[0],), dtype=np.float64)
-    rc = _load().oracle_mla_decode_rows(qb.ctypes.data, kvb.ctypes.data, sl.ctypes.data,
-                                        B, Sq, H, L_max, d_qk, d_v, float(scale),
-                                        rows.ctypes.data, rows.shape[0],
-                                        out.ctypes.data, lse.ctypes.data, int(num_threads))
+    keep, sp = _sinks_arg(sinks, H)
+    rc = _load().oracle_mla_decode_rows_sinks(qb.ctypes.data, kvb.ctypes.data, sl.ctypes.data,
+                                              B, Sq, H, L_max, d_qk, d_v, float(scale), sp,
+                                              rows.ctypes.data, rows.shape[0],
+                                              out.ctypes.data, lse.ctypes.data, int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle_mla_decode_rows failed with code {rc}")
     return out, lse

@@ -21,6 +21,18 @@
  *     out[b,t,h,e] = sum_j exp(s_j - m) * kv[b,j,e] / l                (e < d_v)
  *     lse[b,t,h]   = m + ln(l)                                   (natural log)
  *
+ * Attention sinks (optional).  A sink is one extra logit per head, sigma_h,
+ * in the units of the scaled scores, that enters the softmax denominator and
+ * carries no value.  The TileLang summary lists an attention-sink kernel in
+ * its main-results table (section "主实验", row "Attention Sinks") and notes
+ * in "关键发现" that it is a small change to standard attention; it prints no
+ * formula, so this is the plain reading:
+ *     m   = max(sigma_h, max_j s_j)
+ *     l   = sum_j exp(s_j - m) + exp(sigma_h - m)
+ *     out = sum_j exp(s_j - m) * kv[b,j,e] / l,     lse = m + ln(l)
+ * and an empty sequence gives out = 0, lse = sigma_h.  sigma_h = -inf is the
+ * sink-free definition above, bit for bit.
+ *
  * Keys are the d_qk-wide latent rows (512 latent + 64 rope = 576 for MLA) and
  * the values are the first d_v (= 512) columns of the very same rows.  The Sq
  * query tokens of a sequence all see keys 0..L-1 (no mask between them).  An
@@ -57,14 +69,15 @@ static double bf16_bits_to_double(uint16_t bits)
 }
 
 /* One output row (b, t, h): the definition above, written out. `scores` is a
- * caller-owned scratch array of at least L doubles. */
+ * caller-owned scratch array of at least L doubles; `sink` is sigma_h, or
+ * -INFINITY for no sink. */
 static void attend_one_row(const uint16_t *q_row, const uint16_t *kv_seq,
-                           int64_t L, int64_t d_qk, int64_t d_v, double scale,
+                           int64_t L, int64_t d_qk, int64_t d_v, double scale, double sink,
                            double *scores, double *out_row, double *lse_out)
 {
     if (L <= 0) {
         for (int64_t e = 0; e < d_v; ++e) out_row[e] = 0.0;
-        *lse_out = -INFINITY;
+        *lse_out = sink;
         return;
     }
     /* s_j = scale * <q, k_j> over all d_qk columns (latent + rope). */
@@ -75,16 +88,18 @@ static void attend_one_row(const uint16_t *q_row, const uint16_t *kv_seq,
             dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(k_row[d]);
         scores[j] = scale * dot;
     }
-    /* m = max_j s_j */
+    /* m = max(sink, max_j s_j) */
     double m = scores[0];
     for (int64_t j = 1; j < L; ++j)
         if (scores[j] > m) m = scores[j];
-    /* w_j = exp(s_j - m), l = sum_j w_j */
+    if (sink > m) m = sink;
+    /* w_j = exp(s_j - m), l = sum_j w_j + exp(sink - m) (the sink term is 0 for no sink) */
     double l = 0.0;
     for (int64_t j = 0; j < L; ++j) {
         scores[j] = exp(scores[j] - m);
         l += scores[j];
     }
+    l += exp(sink - m);
     /* out_e = sum_j w_j * v_j[e] / l, with v_j = first d_v columns of row j */
     for (int64_t e = 0; e < d_v; ++e) out_row[e] = 0.0;
     for (int64_t j = 0; j < L; ++j) {
@@ -102,13 +117,14 @@ static void attend_one_row(const uint16_t *q_row, const uint16_t *kv_seq,
  *   q       : bf16 bits, [B, Sq, H, d_qk] contiguous
  *   kv      : bf16 bits, [B, L_max, d_qk] contiguous (values = first d_v cols)
  *   seqlens : int32 [B], 0 <= seqlens[b] <= L_max
+ *   sinks   : double [H] sink logits, or NULL for none
  *   out     : double [B, Sq, H, d_v];  lse : double [B, Sq, H]
  * Returns 0 on success, -1 on bad arguments, -2 on allocation failure.
  */
-int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
-                      int64_t B, int64_t Sq, int64_t H, int64_t L_max,
-                      int64_t d_qk, int64_t d_v, double scale,
-                      double *out, double *lse, int num_threads)
+int oracle_mla_decode_sinks(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                            int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                            int64_t d_qk, int64_t d_v, double scale, const double *sinks,
+                            double *out, double *lse, int num_threads)
 {
     if (!q || !kv || !seqlens || !out || !lse) return -1;
     if (B < 0 || Sq < 1 || H < 1 || L_max < 0 || d_qk < 1 || d_v < 1 || d_v > d_qk) return -1;
@@ -131,8 +147,9 @@ int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seql
 #pragma omp for schedule(dynamic, 1)
             for (int64_t r = 0; r < rows; ++r) {
                 const int64_t b = r / (Sq * H);
+                const double sink = sinks ? sinks[r % H] : -INFINITY;
                 attend_one_row(q + r * d_qk, kv + b * L_max * d_qk, seqlens[b],
-                               d_qk, d_v, scale, scores, out + r * d_v, lse + r);
+                               d_qk, d_v, scale, sink, scores, out + r * d_v, lse + r);
             }
             free(scores);
         }
@@ -140,16 +157,25 @@ int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seql
     return failed ? -2 : 0;
 }
 
+int oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                      int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                      int64_t d_qk, int64_t d_v, double scale,
+                      double *out, double *lse, int num_threads)
+{
+    return oracle_mla_decode_sinks(q, kv, seqlens, B, Sq, H, L_max, d_qk, d_v, scale, NULL, out, lse,
+                                   num_threads);
+}
+
 /*
  * Sampled oracle: the same definition for a caller-chosen list of flattened
  * row indices r = (b * Sq + t) * H + h, so that full-size workloads can be
- * checked row by row.  out is [n_rows, d_v], lse is [n_rows].
+ * checked row by row.  out is [n_rows, d_v], lse is [n_rows]; sinks as above.
  */
-int oracle_mla_decode_rows(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
-                           int64_t B, int64_t Sq, int64_t H, int64_t L_max,
-                           int64_t d_qk, int64_t d_v, double scale,
-                           const int64_t *row_ids, int64_t n_rows,
-                           double *out, double *lse, int num_threads)
+int oracle_mla_decode_rows_sinks(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                                 int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                                 int64_t d_qk, int64_t d_v, double scale, const double *sinks,
+                                 const int64_t *row_ids, int64_t n_rows,
+                                 double *out, double *lse, int num_threads)
 {
     if (!q || !kv || !seqlens || !row_ids || !out || !lse) return -1;
     if (B < 0 || Sq < 1 || H < 1 || L_max < 0 || d_qk < 1 || d_v < 1 || d_v > d_qk) return -1;
@@ -174,13 +200,24 @@ int oracle_mla_decode_rows(const uint16_t *q, const uint16_t *kv, const int32_t 
             for (int64_t i = 0; i < n_rows; ++i) {
                 const int64_t r = row_ids[i];
                 const int64_t b = r / (Sq * H);
+                const double sink = sinks ? sinks[r % H] : -INFINITY;
                 attend_one_row(q + r * d_qk, kv + b * L_max * d_qk, seqlens[b],
-                               d_qk, d_v, scale, scores, out + i * d_v, lse + i);
+                               d_qk, d_v, scale, sink, scores, out + i * d_v, lse + i);
             }
             free(scores);
         }
     }
     return failed ? -2 : 0;
+}
+
+int oracle_mla_decode_rows(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens,
+                           int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                           int64_t d_qk, int64_t d_v, double scale,
+                           const int64_t *row_ids, int64_t n_rows,
+                           double *out, double *lse, int num_threads)
+{
+    return oracle_mla_decode_rows_sinks(q, kv, seqlens, B, Sq, H, L_max, d_qk, d_v, scale, NULL, row_ids,
+                                        n_rows, out, lse, num_threads);
 }
 
 /* Number of OpenMP threads a parallel region of this library would use. */

@@ -233,3 +233,77 @@ def pin_sdpa_library(impl):
 ALL_PINS = [pin_single_key, pin_identical_keys, pin_zero_query, pin_two_keys, pin_rope_shift,
             pin_value_columns, pin_permutation, pin_independence, pin_tail_ignored,
             pin_brute_force_decimal, pin_sdpa_library]
+
+
+# ---------------------------------------------------------------- attention sinks
+# impl(q, kv, seqlens, scale, d_v, sinks) with sinks a float64 [H] array of
+# per-head sink logits (one extra softmax term without a value) or None.
+
+def pin_sink_absent_is_minus_inf(impl):
+    """A sink of -inf adds exp(-inf) = 0 to the denominator and cannot be the
+    max: the result equals the sink-free one."""
+    g = torch.Generator().manual_seed(31)
+    q = _rand_bf16((2, 2, 3, 576), g)
+    kv = _rand_bf16((2, 40, 576), g)
+    sl = np.array([40, 9], np.int32)
+    o0, l0 = impl(q, kv, sl, SCALE, 512, None)
+    o1, l1 = impl(q, kv, sl, SCALE, 512, np.full(3, -np.inf))
+    np.testing.assert_array_equal(o1, o0)
+    np.testing.assert_array_equal(l1, l0)
+
+
+def pin_sink_zero_query(impl):
+    """q = 0: every score is 0, so with sink sigma the weights are 1 / (L + e^sigma)
+    each: out = mean(V) * L / (L + e^sigma) and lse = ln(L + e^sigma).  The
+    sinks span both signs and one far above the scores (e^800 overflows a
+    double, so the sink must take part in the max)."""
+    g = torch.Generator().manual_seed(32)
+    q = torch.zeros((2, 1, 4, 576), dtype=torch.bfloat16)
+    kv = _rand_bf16((2, 30, 576), g)
+    sl = np.array([30, 7], np.int32)
+    sinks = np.array([-3.0, 0.0, 2.5, 800.0])
+    out, lse = impl(q, kv, sl, SCALE, 512, sinks)
+    for b, L in enumerate(sl):
+        mean = kv[b, :L, :512].double().mean(dim=0).numpy()
+        for h, sg in enumerate(sinks):
+            # ln(L + e^sg) and L / (L + e^sg) written to stay finite for sg = 800
+            ref_lse = max(sg, math.log(L)) + math.log1p(math.exp(-abs(sg - math.log(L))))
+            frac = math.exp(math.log(L) - ref_lse)
+            np.testing.assert_allclose(out[b, 0, h], mean * frac, rtol=1e-12, atol=1e-300)
+            assert abs(lse[b, 0, h] - ref_lse) <= 1e-12 * max(1.0, abs(ref_lse))
+
+
+def pin_sink_is_a_value_free_key(impl):
+    """A sink equals one more key whose value is zero: append a row that is 0
+    in the 512 value columns and has rope columns r, and set the sink to that
+    row's score scale * <q_rope, r> (computed exactly in fp64).  The sink
+    result must equal the sink-free result over L + 1 keys.  One query row per
+    case (B = Sq = H = 1), so each case's sink is that row's own score."""
+    g = torch.Generator().manual_seed(33)
+    for case, L in enumerate([1, 5, 64]):
+        q = _rand_bf16((1, 1, 1, 576), g)
+        kv = _rand_bf16((1, L + 1, 576), g)
+        kv[0, L, :512] = 0
+        kv[0, L, 512:] = _rand_bf16((64,), g, sigma=4.0 + case)
+        sigma = SCALE * float(torch.dot(q[0, 0, 0, 512:].double(), kv[0, L, 512:].double()))
+        o_s, l_s = impl(q, kv, np.array([L], np.int32), SCALE, 512, np.array([sigma]))
+        o_k, l_k = impl(q, kv, np.array([L + 1], np.int32), SCALE, 512, None)
+        np.testing.assert_allclose(o_s, o_k, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l_s, l_k, rtol=0, atol=1e-12)
+
+
+def pin_sink_empty_sequence(impl):
+    """L = 0: nothing to attend to; out = 0 and the log-sum-exp is the sink
+    alone."""
+    g = torch.Generator().manual_seed(34)
+    q = _rand_bf16((2, 1, 2, 576), g)
+    kv = _rand_bf16((2, 8, 576), g)
+    sl = np.array([0, 8], np.int32)
+    sinks = np.array([1.25, -7.0])
+    out, lse = impl(q, kv, sl, SCALE, 512, sinks)
+    np.testing.assert_array_equal(out[0], 0.0)
+    np.testing.assert_array_equal(lse[0, 0], sinks)
+
+
+SINK_PINS = [pin_sink_absent_is_minus_inf, pin_sink_zero_query, pin_sink_is_a_value_free_key,
+             pin_sink_empty_sequence]

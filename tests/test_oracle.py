@@ -24,6 +24,28 @@ def test_oracle_pin(pin):
     pin(oracle_impl)
 
 
+def sink_oracle_impl(q, kv, sl, scale, d_v, sinks):
+    return oracle.mla_decode(q, kv, sl, scale, d_v=d_v, sinks=sinks)
+
+
+@pytest.mark.parametrize("pin", pins.SINK_PINS, ids=lambda p: p.__name__)
+def test_oracle_sink_pin(pin):
+    pin(sink_oracle_impl)
+
+
+def test_sink_rows_entry_matches_full():
+    g = torch.Generator().manual_seed(5)
+    q = (torch.randn(2, 2, 3, 576, generator=g)).to(torch.bfloat16)
+    kv = (torch.randn(2, 30, 576, generator=g)).to(torch.bfloat16)
+    sl = np.array([30, 0], np.int32)
+    sinks = np.array([0.5, -1.0, 3.0])
+    out, lse = oracle.mla_decode(q, kv, sl, pins.SCALE, sinks=sinks)
+    rows = np.array([0, 4, 7, 11])
+    o2, l2 = oracle.mla_decode_rows(q, kv, sl, pins.SCALE, rows, sinks=sinks)
+    np.testing.assert_array_equal(o2, out.reshape(-1, 512)[rows])
+    np.testing.assert_array_equal(l2, lse.reshape(-1)[rows])
+
+
 def test_rows_entry_matches_full():
     g = torch.Generator().manual_seed(3)
     q = (torch.randn(3, 2, 5, 576, generator=g)).to(torch.bfloat16)
@@ -66,7 +88,7 @@ def test_golden_fixture_reproduces():
 
 def _np_attention(q, kv, sl, scale, d_v, *, qk_cols=None, v_cols=None, lse_base=math.e,
                   scale_used=True, sign=1.0, len_delta=0, add_max_to_lse=True,
-                  normalise=True, head_mixup=False):
+                  normalise=True, head_mixup=False, sinks=None, sink_mode="correct"):
     qd = q.to(torch.float64).numpy()
     kd = kv.to(torch.float64).numpy()
     B, Sq, H, d = qd.shape
@@ -79,15 +101,24 @@ def _np_attention(q, kv, sl, scale, d_v, *, qk_cols=None, v_cols=None, lse_base=
         L = max(0, min(L, kd.shape[1]))
         for t in range(Sq):
             for h in range(H):
+                sg = -np.inf if sinks is None else float(sinks[0 if sink_mode == "first_head" else h])
+                if sink_mode == "scaled":
+                    sg *= scale
                 if L == 0:
-                    lse[b, t, h] = -np.inf
+                    lse[b, t, h] = -np.inf if (sink_mode == "empty_minus_inf" or sinks is None) else sg
                     continue
                 qrow = qd[b, t, 0 if head_mixup else h]
                 s = sign * (kd[b, :L, qc] @ qrow[qc]) * (scale if scale_used else 1.0)
                 m = s.max()
+                if sink_mode != "not_in_max":
+                    m = max(m, sg)
                 w = np.exp(s - m)
                 l = w.sum()
+                if sink_mode != "ignored":
+                    l += np.exp(sg - m)
                 o = w @ kd[b, :L, vc]
+                if sink_mode == "carries_first_value":
+                    o = o + np.exp(sg - m) * kd[b, 0, vc]
                 out[b, t, h] = o / l if normalise else o
                 lse[b, t, h] = ((m if add_max_to_lse else 0.0) + np.log(l)) / math.log(lse_base)
     return out, lse
@@ -106,6 +137,39 @@ MUTANTS = {
     "output_not_normalised": dict(normalise=False),
     "heads_mixed_up": dict(head_mixup=True),
 }
+
+
+SINK_MUTANTS = {
+    "correct": {},
+    "sink_ignored": dict(sink_mode="ignored"),
+    "sink_multiplied_by_scale": dict(sink_mode="scaled"),
+    "sink_left_out_of_max": dict(sink_mode="not_in_max"),
+    "sink_carries_a_value": dict(sink_mode="carries_first_value"),
+    "first_head_sink_for_all": dict(sink_mode="first_head"),
+    "empty_sequence_lse_minus_inf": dict(sink_mode="empty_minus_inf"),
+}
+
+
+def _run_sink_pins(kwargs):
+    def impl(q, kv, sl, scale, d_v, sinks):
+        return _np_attention(q, kv, sl, scale, d_v, sinks=sinks, **kwargs)
+    failed = []
+    for pin in pins.SINK_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+@pytest.mark.parametrize("name", sorted(SINK_MUTANTS))
+def test_sink_pins_catch_planted_mistakes(name):
+    failed = _run_sink_pins(SINK_MUTANTS[name])
+    if name == "correct":
+        assert failed == [], f"a correct stand-in must pass every sink pin, failed: {failed}"
+    else:
+        assert failed, f"planted mistake '{name}' passed every sink pin"
 
 
 def _run_pins(kwargs):
