@@ -199,8 +199,17 @@ def run_ours(args, w: W.Workload):
     lse = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32, device=dev)
     stream = torch.cuda.Stream(dev)
 
+    # --sinks: the same decode with per-head attention-sink logits (seeded)
+    sinks_d = None
+    if args.sinks:
+        gs = torch.Generator().manual_seed(w.seed + 17)
+        sinks_d = (torch.randn(w.H, generator=gs) * 2.0).to(dev)
+
     def step():
-        M.mla_decode_run(plan, qd, kvd, sld, w.scale, out, lse, ws, stream=stream)
+        if sinks_d is None:
+            M.mla_decode_run(plan, qd, kvd, sld, w.scale, out, lse, ws, stream=stream)
+        else:
+            M.mla_decode_run_sinks(plan, qd, kvd, sld, w.scale, sinks_d, out, lse, ws, stream=stream)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -324,7 +333,8 @@ def run_ours(args, w: W.Workload):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_desc(w), "global_batch": w.B * world, "seq_len": w.L,
+            "config": {"workload": workload_desc(w) + (" + per-head attention sinks" if args.sinks else ""),
+                       "global_batch": w.B * world, "seq_len": w.L,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "kernel": {1: "transposed", 2: "pair"}.get(plan.kernel, str(plan.kernel)),
                        "group_rows": plan.group_rows, "partitions": plan.num_partitions,
@@ -359,6 +369,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="metric", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sinks", action="store_true",
+                    help="time the attention-sink entry point (per-head sink logits) on the same workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -170,6 +170,30 @@ mla_status mla_decode_run_phase(const mla_plan* plan, const void* q, const void*
                                 size_t workspace_bytes, void* stream, int32_t phase);
 
 /*
+ * mla_decode_run_sinks -- mla_decode_run with attention sinks: one extra
+ * logit per head that enters every row's softmax denominator and carries no
+ * value.  "TileLang: Bridging Programmability and Performance in Modern
+ * Neural Kernels" (papernotes.org summary) lists an attention-sink kernel in
+ * its main-results table (section "主实验", row "Attention Sinks") and notes
+ * in "关键发现" that it differs from standard attention by a few lines; the
+ * formula is not printed, and this is its plain reading.  For a row of head h
+ * with scaled scores s_j (j < L) and sink logit sigma_h:
+ *     m = max(sigma_h, max_j s_j),   l = sum_j exp(s_j - m) + exp(sigma_h - m)
+ *     out = sum_j exp(s_j - m) v_j / l,   lse = m + ln l   (natural log)
+ * An empty sequence gives out = 0 and lse = sigma_h.
+ *
+ *   sinks     device, fp32 [H], 4-byte aligned, in the units of the scaled
+ *             scores (it is not multiplied by softmax_scale); the same logits
+ *             apply to every sequence and query token.  NULL = no sinks
+ *             (exactly mla_decode_run); -inf entries switch one head's sink off.
+ * Every other argument, the launches and the return codes are those of
+ * mla_decode_run.
+ */
+mla_status mla_decode_run_sinks(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                                float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
  * mla_decode_check -- synchronize `stream`, read and clear the workspace's
  * device status words.  Returns MLA_OK if no run since the last check
  * recorded a fault, else MLA_ERR_TIMEOUT / MLA_ERR_SEQLEN (the first recorded),

@@ -8,7 +8,7 @@ device is not an sm_100 GPU, the calls raise.
 Entry points mirror include/mla_decode.h:
     mla_decode_plan, mla_decode_workspace_init, mla_decode_run,
     mla_decode_check, mla_status_string, mla_decode_set_debug,
-    mla_decode_run_noalloc
+    mla_decode_run_noalloc, mla_decode_run_sinks
 plus the convenience wrappers ``mla_decode`` (device tensors in, device
 tensors out) and ``mla_decode_host`` (host tensors in and out, with the
 copies done here around the library call).
@@ -35,7 +35,7 @@ MLA_KERNEL_PAIR = 2
 MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
 EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
-                    "mla_decode_check", "mla_decode_run_noalloc",
+                    "mla_decode_check", "mla_decode_run_noalloc", "mla_decode_run_sinks",
                     "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug")
 
 
@@ -90,6 +90,9 @@ def load_library(build_if_missing: bool = True):
         lib.mla_decode_run.restype = c_i32
         lib.mla_decode_run.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp, c_sz,
                                        c_vp]
+        lib.mla_decode_run_sinks.restype = c_i32
+        lib.mla_decode_run_sinks.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp, c_vp,
+                                             c_sz, c_vp]
         lib.mla_decode_run_phase.restype = c_i32
         lib.mla_decode_run_phase.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp,
                                              c_sz, c_vp, c_i32]
@@ -180,6 +183,27 @@ def mla_decode_run(plan: mla_plan, q: torch.Tensor, kv: torch.Tensor, seqlens: t
                                        workspace.numel(), _stream_handle(stream))
     if rc != MLA_OK:
         raise MlaError(rc, "mla_decode_run")
+
+
+def mla_decode_run_sinks(plan: mla_plan, q: torch.Tensor, kv: torch.Tensor, seqlens: torch.Tensor,
+                         softmax_scale: float, sinks: Optional[torch.Tensor], out: torch.Tensor, lse: torch.Tensor,
+                         workspace: torch.Tensor, stream=None) -> None:
+    """mla_decode_run with per-head attention-sink logits: sinks is a CUDA
+    fp32 tensor [H] (units of the scaled scores) or None for no sinks."""
+    B, Sq, H, L = plan.B, plan.Sq, plan.H, plan.L_max
+    _check_tensor(q, "q", torch.bfloat16, (B, Sq, H, D_QK))
+    _check_tensor(kv, "kv", torch.bfloat16, (B, L, D_QK))
+    _check_tensor(seqlens, "seqlens", torch.int32, (B,))
+    _check_tensor(out, "out", torch.bfloat16, (B, Sq, H, D_V))
+    _check_tensor(lse, "lse", torch.float32, (B, Sq, H))
+    if sinks is not None:
+        _check_tensor(sinks, "sinks", torch.float32, (H,))
+    rc = load_library().mla_decode_run_sinks(ctypes.byref(plan), q.data_ptr(), kv.data_ptr(), seqlens.data_ptr(),
+                                             float(softmax_scale), sinks.data_ptr() if sinks is not None else None,
+                                             out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                             workspace.numel(), _stream_handle(stream))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mla_decode_run_sinks")
 
 
 def mla_decode_run_phase(plan: mla_plan, q: torch.Tensor, kv: torch.Tensor, seqlens: torch.Tensor,

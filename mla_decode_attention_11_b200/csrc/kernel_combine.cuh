@@ -3,11 +3,13 @@
 // For a sequence whose KV tiles were cut across k > 1 partitions, partition
 // pieces left (O_s / l_s, lse_s) in fp32.  The merged result is
 //     lse = ln sum_s exp(lse_s),      out = sum_s exp(lse_s - lse) * (O_s / l_s)
-// which is exactly the softmax over the union of the pieces' keys.  The pages
+// which is exactly the softmax over the union of the pieces' keys.  A
+// per-head attention sink (one more softmax term without a value) enters the
+// merged lse only, once per row.  The pages
 // do not describe splitting; this is the standard identity for merging
 // softmax-normalised partial results.  Sequences that were not cut were
 // finished by the main kernel and are skipped; empty sequences (L = 0) are
-// written here as out = 0, lse = -inf.
+// written here as out = 0, lse = -inf (or the head's sink logit).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -27,6 +29,8 @@ struct CombineArgs {
     float* lse;
     const float* part_o;
     const float* part_lse;
+    const float* sinks;  // [H] per-head attention-sink logits (natural-log units), or null
+    int H;
 };
 
 // One warp per query row, 8 rows per CTA.  The kernel is bound by the bytes of
@@ -69,11 +73,13 @@ __global__ void __launch_bounds__(kCombineThreads)
     const size_t orow = static_cast<size_t>(b) * args.R + r;
     const int L = clamp_len(args.seqlens[b], args.L_max, nullptr);
     const long long n = num_tiles(L);
+    // a per-head sink is one more softmax term without a value (-inf: none)
+    const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
     if (n == 0) {
         uint4* dst = reinterpret_cast<uint4*>(args.out + orow * kDv);  // 64 x 16 bytes
         dst[lane] = make_uint4(0u, 0u, 0u, 0u);
         dst[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
-        if (lane == 0) args.lse[orow] = -INFINITY;
+        if (lane == 0) args.lse[orow] = sink;  // nothing to attend to: the sink alone
         return;
     }
     const long long T = (tot + args.P - 1) / args.P;
@@ -90,10 +96,12 @@ __global__ void __launch_bounds__(kCombineThreads)
     for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    m = fmaxf(m, sink);
     float sum = 0.f;
     for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    sum += expf(sink - m);
     const float lse_all = m + logf(sum);
 
     // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v

@@ -536,9 +536,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             redsum[L_id] = l_part;
             ok = group_barrier();
             if (!ok) break;
-            const float l_row = l_part + redsum[L_id ^ 64];
-            const float inv_l = 1.f / l_row;
             const int qrow = g * 128 + static_cast<int>(rank) * 64 + r;  // row within the sequence
+            float l_row = l_part + redsum[L_id ^ 64];
+            // a sink applies once per row: to whole sequences here, to cut ones in the combine
+            float o_fac = 1.f;
+            if (args.sinks != nullptr && pc.slot < 0)
+                o_fac = fold_sink(m_ref, l_row, args.sinks[qrow % args.H] * kLog2e);
+            const float inv_l = o_fac / l_row;
             // O / l leaves TMEM 64 columns at a time and is transposed through a
             // warp-private 32 x 64 fp32 stage, so that each store instruction
             // writes whole row segments (a thread holds one row, and direct

@@ -57,7 +57,25 @@ struct MainArgs {
     unsigned long long timeout_ns;
     int stall_unit;   // test hook: skip this TMA unit in CTA 0 (-1 = off)
     int prefetch_tiles;  // KV tiles to prefetch into L2 ahead of the loads (0 = off)
+    const float* sinks;  // [H] per-head attention-sink logits (natural-log units), or null
+    int H;               // heads: query row r of a sequence belongs to head r % H
 };
+
+// Folds a per-head attention sink into a finished row.  (m, l) are the row's
+// base-2 reference max and sum over its keys, s2 the sink in base-2 units
+// (-inf: no sink).  The sink is one more softmax term without a value:
+// afterwards m = max(m, s2) and l = l 2^(m_old - m) + 2^(s2 - m), and the
+// returned factor 2^(m_old - m) rescales the row's O before it is divided
+// by the new l.
+__device__ __forceinline__ float fold_sink(float& m, float& l, float s2) {
+    const float mn = fmaxf(m, s2);
+    const float c = exp2f(m - mn);
+    l = l * c + exp2f(s2 - mn);
+    m = mn;
+    return c;
+}
+
+constexpr float kLog2e = 1.4426950408889634074f;
 
 template <int G>
 struct TransposedCfg {
@@ -535,11 +553,30 @@ __global__ void __launch_bounds__(192, 1)
             }
             ok = group_barrier();
             if (!ok) break;
-            float inv_l[G];
-#pragma unroll
-            for (int j = 0; j < G; ++j)
-                inv_l[j] = 1.f / (redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j]);
             const int row_base = g * G;  // first query row of this group within the sequence
+            // a sink applies once per row: to whole sequences here, to cut ones in the combine
+            const bool sink_here = (args.sinks != nullptr) && (pc.slot < 0);
+            // thread j < G finishes query row j (sum, sink, lse) and leaves its
+            // 1 / l in the max buffer the piece's last tile did not use
+            float* fin = red + (tile_cnt & 1) * 4 * G;
+            if (row_in_tile < G) {
+                const int j = row_in_tile;
+                float mj = 0.f;
+#pragma unroll
+                for (int jj = 0; jj < G; ++jj)
+                    if (jj == j) mj = m_ref[jj];
+                float lj = redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j];
+                float c = 1.f;
+                if (sink_here) c = fold_sink(mj, lj, args.sinks[(row_base + j) % args.H] * kLog2e);
+                fin[j] = c / lj;
+                const float lse_nat = (mj + log2f(lj)) * 0.69314718055994530942f;
+                if (pc.slot < 0)
+                    args.lse[static_cast<size_t>(pc.b) * args.R + row_base + j] = lse_nat;
+                else
+                    args.part_lse[static_cast<size_t>(pc.slot) * args.R + row_base + j] = lse_nat;
+            }
+            ok = group_barrier();
+            if (!ok) break;
 #pragma unroll
             for (int blk = 0; blk < 4; ++blk) {
                 const int dv = blk * 128 + row_in_tile;
@@ -552,31 +589,16 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const size_t orow = static_cast<size_t>(pc.b) * args.R + row_base + c0 + j;
-                            args.out[orow * kDv + dv] = __float2bfloat16_rn(__uint_as_float(r[j]) * inv_l[c0 + j]);
+                            args.out[orow * kDv + dv] = __float2bfloat16_rn(__uint_as_float(r[j]) * fin[c0 + j]);
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const size_t orow = static_cast<size_t>(pc.slot) * args.R + row_base + c0 + j;
-                            args.part_o[orow * kDv + dv] = __uint_as_float(r[j]) * inv_l[c0 + j];
+                            args.part_o[orow * kDv + dv] = __uint_as_float(r[j]) * fin[c0 + j];
                         }
                     }
                 }
-            }
-            if (row_in_tile < G) {
-                const int j = row_in_tile;
-                float mj = 0.f, lj = 0.f;
-#pragma unroll
-                for (int jj = 0; jj < G; ++jj)
-                    if (jj == j) {
-                        mj = m_ref[jj];
-                    }
-                lj = redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j];
-                const float lse_nat = (mj + log2f(lj)) * 0.69314718055994530942f;
-                if (pc.slot < 0)
-                    args.lse[static_cast<size_t>(pc.b) * args.R + row_base + j] = lse_nat;
-                else
-                    args.part_lse[static_cast<size_t>(pc.slot) * args.R + row_base + j] = lse_nat;
             }
             ptx::tc_fence_before();
             // the next piece reuses the sums buffer only after everyone read it

@@ -228,8 +228,8 @@ mla_status mla_decode_workspace_init(const mla_plan* plan, void* workspace, size
 namespace {
 
 mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
-                      float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
-                      void* stream_, int phases) {
+                      float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream_, int phases) {
     if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
     if (!plan || !q || !kv || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
@@ -246,7 +246,8 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     } else {
         return MLA_ERR_INVALID_ARG;
     }
-    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4))
+    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
+        !aligned(sinks, 4))
         return MLA_ERR_ALIGNMENT;
     const Layout lay = workspace_layout(pl.num_partitions, R);
     if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
@@ -300,6 +301,8 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     a.timeout_ns = tmo ? tmo : kDefaultTimeoutNs;
     a.stall_unit = g_stall_unit.load();
     a.prefetch_tiles = pl.l2_prefetch_tiles;
+    a.sinks = sinks;
+    a.H = pl.H;
 
     if (phases & 1) {
         mla_status st;
@@ -324,6 +327,8 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     c.lse = lse;
     c.part_o = a.part_o;
     c.part_lse = a.part_lse;
+    c.sinks = sinks;
+    c.H = pl.H;
     const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) /
                                                                         mla::kCombineRowsPerCta));
     mla::mla_decode_combine_kernel<<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
@@ -338,14 +343,21 @@ extern "C" {
 mla_status mla_decode_run(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
                           float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                           void* stream) {
-    return run_phases(plan, q, kv, seqlens, softmax_scale, out, lse, workspace, workspace_bytes, stream, 3);
+    return run_phases(plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, workspace, workspace_bytes, stream, 3);
+}
+
+mla_status mla_decode_run_sinks(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                                float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+    return run_phases(plan, q, kv, seqlens, softmax_scale, sinks, out, lse, workspace, workspace_bytes, stream, 3);
 }
 
 mla_status mla_decode_run_phase(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
                                 float softmax_scale, void* out, float* lse, void* workspace, size_t workspace_bytes,
                                 void* stream, int32_t phase) {
     if (phase != 1 && phase != 2) return MLA_ERR_INVALID_ARG;
-    return run_phases(plan, q, kv, seqlens, softmax_scale, out, lse, workspace, workspace_bytes, stream, phase);
+    return run_phases(plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, workspace, workspace_bytes, stream,
+                      phase);
 }
 
 mla_status mla_decode_check(const mla_plan* plan, void* workspace, void* stream) {
@@ -436,7 +448,8 @@ mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const voi
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }
-    st = run_phases(plan, q, kv, seqlens, softmax_scale, out, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES, stream_, 3);
+    st = run_phases(plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES,
+                    stream_, 3);
     if (st != MLA_OK || !wait_and_check) return st;
     if (cudaStreamSynchronize(stream) != cudaSuccess) {
         cudaGetLastError();
