@@ -192,7 +192,10 @@ def run_ours(args, w: W.Workload):
 
     q, kv, sl = W.generate(w, tail_fill=0.0)
     qd, kvd, sld = q.to(dev), kv.to(dev), sl.to(dev)
-    plan = M.mla_decode_plan(w.B, w.Sq, w.H, w.L, device=local)
+    if args.batch_invariant is not None:
+        plan = M.mla_decode_plan_batch_invariant(w.B, w.Sq, w.H, w.L, device=local, split_tiles=args.batch_invariant)
+    else:
+        plan = M.mla_decode_plan(w.B, w.Sq, w.H, w.L, device=local)
     ws = M.alloc_workspace(plan, device=dev)
     M.mla_decode_workspace_init(plan, ws)
     out = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16, device=dev)
@@ -333,7 +336,8 @@ def run_ours(args, w: W.Workload):
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_desc(w) + (" + per-head attention sinks" if args.sinks else ""),
+            "config": {"workload": workload_desc(w) + (" + per-head attention sinks" if args.sinks else "")
+                       + (f" + batch-invariant plan ({plan.split_tiles}-tile chunks)" if plan.split_tiles else ""),
                        "global_batch": w.B * world, "seq_len": w.L,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "kernel": {1: "transposed", 2: "pair"}.get(plan.kernel, str(plan.kernel)),
@@ -369,6 +373,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="metric", choices=sorted(W.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch-invariant", type=int, default=None, metavar="SPLIT_TILES",
+                    help="use the batch-invariant plan, sequences cut every SPLIT_TILES KV tiles (0 = default)")
     ap.add_argument("--sinks", action="store_true",
                     help="time the attention-sink entry point (per-head sink logits) on the same workload")
     args = ap.parse_args()

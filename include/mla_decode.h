@@ -83,7 +83,9 @@ typedef struct mla_plan {
     uint64_t workspace_bytes;  /* bytes the caller must provide to mla_decode_run */
     int32_t l2_prefetch_tiles; /* KV tiles the loader prefetches into L2 ahead of its shared-memory
                                   loads (0..16; a tuning knob, does not change results) */
-    int32_t reserved32;
+    int32_t split_tiles;       /* 0: balanced split-KV schedule (where a sequence is cut depends on the
+                                  whole batch); > 0: batch-invariant schedule, every sequence cut into
+                                  chunks of this many tiles (mla_decode_plan_batch_invariant) */
     uint64_t reserved[5];
 } mla_plan;
 
@@ -123,6 +125,34 @@ mla_status mla_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int3
 mla_status mla_decode_plan_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
                                   int32_t num_partitions_override, int32_t kernel, mla_plan* plan,
                                   size_t* workspace_bytes);
+
+/*
+ * mla_decode_plan_batch_invariant -- a plan whose results do not depend on
+ * the rest of the batch: a sequence's out and lse are bitwise the same
+ * whatever other sequences (and how many) share the call.  The qingkeai.online
+ * essay on TileLang in the DeepSeek-V4 report (section "V4 设计报告里的几个点",
+ * its third point on precision and bitwise alignment) stresses batch
+ * invariance of kernels for uses such as RL; it gives no schedule, and this
+ * is one.  The balanced schedule of mla_decode_plan cuts the flattened KV
+ * tiles of the whole batch into equal ranges, so where a sequence is cut (and
+ * hence the rounding of its partials and their merge) depends on the other
+ * sequences.  Here every sequence is cut into chunks of split_tiles KV tiles
+ * (128 keys each; its last chunk shorter) at fixed offsets from its start;
+ * each chunk is processed on its own and the chunks are merged in order, so
+ * only the placement of work on the GPU depends on the batch.
+ *
+ *   split_tiles  tiles per chunk, 1 <= split_tiles <= 131072; 0 = 16 (2048
+ *                keys).  Sequences of at most split_tiles tiles are computed
+ *                whole.  Smaller chunks spread one long sequence over more
+ *                SMs; larger ones write fewer partials.
+ * Other arguments and return codes as mla_decode_plan (no partition
+ * override: the partition count only places chunks).  The workspace holds one
+ * partial per chunk of B sequences of L_max keys.  Run with mla_decode_run,
+ * mla_decode_run_sinks or mla_decode_run_noalloc (if the workspace fits its
+ * scratch).  For a given split_tiles, kernel choice depends only on Sq * H.
+ */
+mla_status mla_decode_plan_batch_invariant(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                                           int32_t split_tiles, mla_plan* plan, size_t* workspace_bytes);
 
 /*
  * mla_decode_workspace_init -- zero the workspace's status words on `stream`

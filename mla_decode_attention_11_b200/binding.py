@@ -34,7 +34,7 @@ MLA_KERNEL_TRANSPOSED = 1
 MLA_KERNEL_PAIR = 2
 MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
-EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
+EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_plan_batch_invariant", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
                     "mla_decode_check", "mla_decode_run_noalloc", "mla_decode_run_sinks",
                     "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug")
 
@@ -51,7 +51,7 @@ class mla_plan(ctypes.Structure):
                 ("group_rows", ctypes.c_int32), ("num_groups", ctypes.c_int32),
                 ("num_partitions", ctypes.c_int32), ("tile_kv", ctypes.c_int32), ("cta_threads", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
-                ("l2_prefetch_tiles", ctypes.c_int32), ("reserved32", ctypes.c_int32),
+                ("l2_prefetch_tiles", ctypes.c_int32), ("split_tiles", ctypes.c_int32),
                 ("reserved", ctypes.c_uint64 * 5)]
 
     def as_dict(self):
@@ -85,6 +85,9 @@ def load_library(build_if_missing: bool = True):
         lib.mla_decode_plan_kernel.restype = c_i32
         lib.mla_decode_plan_kernel.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
                                                ctypes.POINTER(mla_plan), ctypes.POINTER(c_sz)]
+        lib.mla_decode_plan_batch_invariant.restype = c_i32
+        lib.mla_decode_plan_batch_invariant.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                                        ctypes.POINTER(mla_plan), ctypes.POINTER(c_sz)]
         lib.mla_decode_workspace_init.restype = c_i32
         lib.mla_decode_workspace_init.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_sz, c_vp]
         lib.mla_decode_run.restype = c_i32
@@ -140,6 +143,22 @@ def mla_decode_plan(B: int, Sq: int, H: int, L_max: int, device: Optional[int] =
                                  ctypes.byref(p), ctypes.byref(ws))
     if rc != MLA_OK:
         raise MlaError(rc, "mla_decode_plan")
+    return p
+
+
+def mla_decode_plan_batch_invariant(B: int, Sq: int, H: int, L_max: int, device: Optional[int] = None,
+                                    split_tiles: int = 0) -> mla_plan:
+    """A plan whose per-sequence results are bitwise independent of the rest of
+    the batch: every sequence is cut into chunks of split_tiles KV tiles
+    (0 = the library default) at fixed offsets (mla_decode_plan_batch_invariant)."""
+    if device is None:
+        device = torch.cuda.current_device()
+    p = mla_plan()
+    ws = ctypes.c_size_t(0)
+    rc = load_library().mla_decode_plan_batch_invariant(int(B), int(Sq), int(H), int(L_max), int(device),
+                                                        int(split_tiles), ctypes.byref(p), ctypes.byref(ws))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mla_decode_plan_batch_invariant")
     return p
 
 

@@ -31,6 +31,7 @@ struct CombineArgs {
     const float* part_lse;
     const float* sinks;  // [H] per-head attention-sink logits (natural-log units), or null
     int H;
+    int split_tiles;     // 0: balanced schedule; > 0: batch-invariant chunks of this many tiles
 };
 
 // One warp per query row, 8 rows per CTA.  The kernel is bound by the bytes of
@@ -47,10 +48,10 @@ __global__ void __launch_bounds__(kCombineThreads)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // flat tile offset of sequence b, and the total
+    // flat unit offset of sequence b, and the total (units: tiles, or S-tile chunks)
     long long acc = 0, tot = 0;
     for (int i = threadIdx.x; i < args.B; i += kCombineThreads) {
-        const long long n = num_tiles(clamp_len(args.seqlens[i], args.L_max, nullptr));
+        const long long n = num_units(clamp_len(args.seqlens[i], args.L_max, nullptr), args.split_tiles);
         tot += n;
         if (i < b) acc += n;
     }
@@ -72,7 +73,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     if (r >= args.R) return;
     const size_t orow = static_cast<size_t>(b) * args.R + r;
     const int L = clamp_len(args.seqlens[b], args.L_max, nullptr);
-    const long long n = num_tiles(L);
+    const long long n = num_units(L, args.split_tiles);
     // a per-head sink is one more softmax term without a value (-inf: none)
     const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
     if (n == 0) {
@@ -82,14 +83,24 @@ __global__ void __launch_bounds__(kCombineThreads)
         if (lane == 0) args.lse[orow] = sink;  // nothing to attend to: the sink alone
         return;
     }
-    const long long T = (tot + args.P - 1) / args.P;
-    const int p0 = static_cast<int>(acc / T);
-    const int p1 = static_cast<int>((acc + n - 1) / T);
-    if (p0 == p1) return;  // finished by the main kernel
-    const int k = p1 - p0 + 1;
+    int k, p0 = 0;
+    if (args.split_tiles > 0) {
+        // batch-invariant chunks: chunk i of b is in slot acc + i
+        if (n == 1) return;  // one chunk: finished by the main kernel
+        k = static_cast<int>(n);
+    } else {
+        const long long T = (tot + args.P - 1) / args.P;
+        p0 = static_cast<int>(acc / T);
+        const int p1 = static_cast<int>((acc + n - 1) / T);
+        if (p0 == p1) return;  // finished by the main kernel
+        k = p1 - p0 + 1;
+    }
     // slot of the i-th piece: the first partition's piece continues after it
     // (2 p0 + 1), every later piece started before its partition (2 p)
-    auto slot_of = [&](int i) { return (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i); };
+    auto slot_of = [&](int i) {
+        if (args.split_tiles > 0) return static_cast<int>(acc) + i;
+        return (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i);
+    };
 
     // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
     float m = -INFINITY;

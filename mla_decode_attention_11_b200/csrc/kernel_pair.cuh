@@ -159,11 +159,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         ptx::tmem_relinquish_pair();
     }
     if (warp == 0) {
-        const long long total = total_tiles_warp(args.seqlens, args.B, args.L_max);
+        const long long total = total_units_warp(args.seqlens, args.B, args.L_max, args.split_tiles);
         const long long T = (total + args.P - 1) / args.P;
         int bf;
         long long af;
-        locate_warp(args.seqlens, args.B, args.L_max, static_cast<long long>(p) * T, &bf, &af);
+        locate_warp(args.seqlens, args.B, args.L_max, args.split_tiles, static_cast<long long>(p) * T, &bf, &af);
         if (lane == 0) {
             *b_first_slot = bf;
             *acc_first_slot = af;
@@ -191,6 +191,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         walker.B = args.B;
         walker.L_max = args.L_max;
         walker.p = p;
+        walker.S = args.split_tiles;
+        walker.k = 0;
         walker.start = static_cast<long long>(p) * T;
         walker.end = walker.start + T < total ? walker.start + T : total;
         walker.b = smem_ok ? *b_first_slot : args.B;  // misaligned smem: do nothing
@@ -211,17 +213,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             // is prefetched whole (all 128 rows, K and V columns alike); on
             // entering a later piece the cursor also prefetches that piece's
             // Q rows, so the Q reload after a piece boundary hits L2.  The two
-            // CTAs split the column chunks.
+            // CTAs split the column chunks.  The cursor starts after the first
+            // piece's Q loads are out and skips the first tile (loaded at once),
+            // so nothing queues ahead of the loads the first MMA needs.
             PieceWalker pf_walker = walker;
-            Piece pf_pc;
-            bool pf_live = args.prefetch_tiles > 0 && pf_walker.next(pf_pc);
-            int pf_t = pf_live ? pf_pc.tile_lo : 0;
-            auto prefetch_next = [&]() {
+            Piece pf_pc{};
+            bool pf_live = false, pf_started = false;
+            int pf_t = 0;
+            auto prefetch_next = [&](bool issue) {
                 if (!pf_live) return;
                 int row0 = pf_t * kTileKV;
                 if (row0 + kTileKV > pf_pc.L) row0 = pf_pc.L - kTileKV;
-                for (int j = static_cast<int>(rank); j < kNumChunks; j += 2)
-                    ptx::tma_prefetch_3d(&tm_v, j * kChunk, row0, pf_pc.b);
+                if (issue)
+                    for (int j = static_cast<int>(rank); j < kNumChunks; j += 2)
+                        ptx::tma_prefetch_3d(&tm_v, j * kChunk, row0, pf_pc.b);
                 if (++pf_t == pf_pc.tile_hi) {
                     pf_live = pf_walker.next(pf_pc);
                     if (pf_live) {
@@ -231,7 +236,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                     }
                 }
             };
-            for (int i = 0; i < args.prefetch_tiles; ++i) prefetch_next();
             Piece pc;
             while (ok && walker.next(pc)) {
                 if (piece_cnt > 0) ok = ptx::mbar_wait_bounded(q_empty, (piece_cnt - 1) & 1, tmo);
@@ -243,7 +247,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                         ptx::tma_load_2d_pair(q_smem + c * C::kQChunk, &tm_q, lead_q_full, c * kChunk, qrow);
                 ++unit;
                 for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
-                    prefetch_next();
+                    if (!pf_started) {
+                        pf_started = true;
+                        pf_live = args.prefetch_tiles > 0 && pf_walker.next(pf_pc);
+                        pf_t = pf_live ? pf_pc.tile_lo : 0;
+                        prefetch_next(false);  // this tile: loaded now
+                        for (int i = 1; i < args.prefetch_tiles; ++i) prefetch_next(true);
+                    }
+                    prefetch_next(true);
                     int row0 = t * kTileKV;
                     if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;
                     const int krow = row0 + static_cast<int>(rank) * 64;

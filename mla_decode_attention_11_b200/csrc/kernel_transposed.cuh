@@ -59,6 +59,7 @@ struct MainArgs {
     int prefetch_tiles;  // KV tiles to prefetch into L2 ahead of the loads (0 = off)
     const float* sinks;  // [H] per-head attention-sink logits (natural-log units), or null
     int H;               // heads: query row r of a sequence belongs to head r % H
+    int split_tiles;     // 0: balanced schedule; > 0: batch-invariant chunks of this many tiles
 };
 
 // Folds a per-head attention sink into a finished row.  (m, l) are the row's
@@ -221,12 +222,12 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (warp == 0) {
         // partition bounds in the flat tile space, and the first sequence
-        const long long total = total_tiles_warp(args.seqlens, args.B, args.L_max);
+        const long long total = total_units_warp(args.seqlens, args.B, args.L_max, args.split_tiles);
         const long long T = (total + args.P - 1) / args.P;
         const long long start = static_cast<long long>(p) * T;
         int bf;
         long long af;
-        locate_warp(args.seqlens, args.B, args.L_max, start, &bf, &af);
+        locate_warp(args.seqlens, args.B, args.L_max, args.split_tiles, start, &bf, &af);
         if (lane == 0) {
             *b_first_slot = bf;
             *acc_first_slot = af;
@@ -253,6 +254,8 @@ __global__ void __launch_bounds__(192, 1)
         walker.B = args.B;
         walker.L_max = args.L_max;
         walker.p = p;
+        walker.S = args.split_tiles;
+        walker.k = 0;
         walker.start = static_cast<long long>(p) * T;
         walker.end = walker.start + T < total ? walker.start + T : total;
         walker.b = *b_first_slot;

@@ -54,11 +54,21 @@ struct Layout {
     size_t part_lse_off, part_o_off, total;
 };
 
-Layout workspace_layout(int P, int R) {
+// partial slots: 2 per partition (balanced schedule), or one per S-tile chunk
+// of every sequence at its longest (batch-invariant schedule)
+long long num_slots(const mla_plan& pl) {
+    if (pl.split_tiles > 0) {
+        const long long tiles = (static_cast<long long>(pl.L_max) + mla::kTileKV - 1) / mla::kTileKV;
+        return static_cast<long long>(pl.B) * ((tiles + pl.split_tiles - 1) / pl.split_tiles);
+    }
+    return 2LL * pl.num_partitions;
+}
+
+Layout workspace_layout(long long slots, int R) {
     Layout l;
     l.part_lse_off = kHeaderBytes;
-    l.part_o_off = align_up(l.part_lse_off + size_t(2) * P * R * sizeof(float), 256);
-    l.total = l.part_o_off + size_t(2) * P * R * mla::kDv * sizeof(float);
+    l.part_o_off = align_up(l.part_lse_off + size_t(slots) * R * sizeof(float), 256);
+    l.total = l.part_o_off + size_t(slots) * R * mla::kDv * sizeof(float);
     return l;
 }
 
@@ -98,6 +108,7 @@ constexpr int kPairNV = MLA_PAIR_NV;
 constexpr int kPairNS = MLA_PAIR_NS;
 constexpr int kPairNP = MLA_PAIR_NP;  // P buffers in shared memory
 constexpr int kDefaultPrefetchTiles = 1;
+constexpr int kDefaultSplitTiles = 16;  // batch-invariant chunks: 16 tiles = 2048 keys
 using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS, kPairNP>;
 
 mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
@@ -207,7 +218,23 @@ mla_status mla_decode_plan_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_ma
     p.num_partitions = P;
     p.tile_kv = mla::kTileKV;
     p.l2_prefetch_tiles = kDefaultPrefetchTiles;
-    p.workspace_bytes = workspace_layout(P, R).total;
+    p.split_tiles = 0;
+    p.workspace_bytes = workspace_layout(num_slots(p), R).total;
+    *plan = p;
+    if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
+    return MLA_OK;
+}
+
+mla_status mla_decode_plan_batch_invariant(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                                           int32_t split_tiles, mla_plan* plan, size_t* workspace_bytes) {
+    if (!plan) return MLA_ERR_INVALID_ARG;
+    if (split_tiles == 0) split_tiles = kDefaultSplitTiles;
+    if (split_tiles < 1 || split_tiles > (1 << 17)) return MLA_ERR_INVALID_ARG;
+    mla_plan p;
+    const mla_status st = mla_decode_plan_kernel(B, Sq, H, L_max, device, 0, 0, &p, nullptr);
+    if (st != MLA_OK) return st;
+    p.split_tiles = split_tiles;
+    p.workspace_bytes = workspace_layout(num_slots(p), Sq * H).total;
     *plan = p;
     if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
     return MLA_OK;
@@ -239,6 +266,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
         pl.group_rows * pl.num_groups != R)
         return MLA_ERR_INVALID_ARG;
     if (pl.l2_prefetch_tiles < 0 || pl.l2_prefetch_tiles > 16) return MLA_ERR_INVALID_ARG;
+    if (pl.split_tiles < 0 || pl.split_tiles > (1 << 17)) return MLA_ERR_INVALID_ARG;
     if (pl.kernel == MLA_KERNEL_TRANSPOSED) {
         if (pl.group_rows != 16 && pl.group_rows != 32) return MLA_ERR_INVALID_ARG;
     } else if (pl.kernel == MLA_KERNEL_PAIR) {
@@ -249,7 +277,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
         !aligned(sinks, 4))
         return MLA_ERR_ALIGNMENT;
-    const Layout lay = workspace_layout(pl.num_partitions, R);
+    const Layout lay = workspace_layout(num_slots(pl), R);
     if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
 
     int dev = -1;
@@ -303,6 +331,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     a.prefetch_tiles = pl.l2_prefetch_tiles;
     a.sinks = sinks;
     a.H = pl.H;
+    a.split_tiles = pl.split_tiles;
 
     if (phases & 1) {
         mla_status st;
@@ -329,6 +358,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     c.part_lse = a.part_lse;
     c.sinks = sinks;
     c.H = pl.H;
+    c.split_tiles = pl.split_tiles;
     const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) /
                                                                         mla::kCombineRowsPerCta));
     mla::mla_decode_combine_kernel<<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
@@ -430,7 +460,9 @@ mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const voi
     if (!plan) return MLA_ERR_INVALID_ARG;
     if (plan->num_partitions < 1 || plan->num_partitions > 4096 || plan->Sq < 1 || plan->H < 1)
         return MLA_ERR_INVALID_ARG;
-    const size_t need = workspace_layout(plan->num_partitions, plan->Sq * plan->H).total;
+    if (plan->split_tiles < 0 || plan->split_tiles > (1 << 17) || plan->B < 1 || plan->L_max < 1)
+        return MLA_ERR_INVALID_ARG;
+    const size_t need = workspace_layout(num_slots(*plan), plan->Sq * plan->H).total;
     if (need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {

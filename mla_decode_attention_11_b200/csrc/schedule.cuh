@@ -15,6 +15,17 @@
 // in p and continues after it).  Both can occur in one partition, for two
 // different sequences; a sequence that both starts before and ends after p is
 // p's only sequence and uses 2p.
+//
+// Batch-invariant schedule (S > 0 tiles).  Where a sequence is cut above
+// depends on every other sequence of the batch, and so do the rounding of
+// its partials and of their merge.  With S > 0 the unit of work is instead a
+// chunk of S tiles of one sequence (its last chunk shorter): chunk k of
+// sequence b covers tiles [kS, min(kS + S, n_b)), is always a piece of its
+// own, and a sequence of u_b > 1 chunks writes chunk k to slot acc_b + k
+// (acc_b = chunks of the sequences before b).  The flat list of chunks is cut
+// into P equal ranges as before; only which CTA computes a chunk depends on
+// the batch, not what it computes, so a sequence's output is bitwise the same
+// in any batch.
 #pragma once
 
 #include <cstdint>
@@ -41,6 +52,12 @@ __device__ __forceinline__ int clamp_len(int L, int L_max, uint32_t* status) {
 
 __device__ __forceinline__ int num_tiles(int L) { return (L + kTileKV - 1) / kTileKV; }
 
+// schedule units of a sequence of L keys: its tiles (S = 0) or its S-tile chunks
+__device__ __forceinline__ long long num_units(int L, int S) {
+    const long long n = num_tiles(L);
+    return S > 0 ? (n + S - 1) / S : n;
+}
+
 // Warp-cooperative: total tiles over all sequences, and (for `start`) the
 // first sequence whose tiles reach past `start` with its flat offset.
 // Every lane returns the same values.
@@ -56,21 +73,21 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
     return v;
 }
 
-__device__ inline long long total_tiles_warp(const int32_t* seqlens, int B, int L_max) {
+__device__ inline long long total_units_warp(const int32_t* seqlens, int B, int L_max, int S) {
     const int lane = threadIdx.x & 31;
     long long s = 0;
-    for (int b = lane; b < B; b += 32) s += num_tiles(clamp_len(seqlens[b], L_max, nullptr));
+    for (int b = lane; b < B; b += 32) s += num_units(clamp_len(seqlens[b], L_max, nullptr), S);
     return warp_sum_ll(s);
 }
 
-// Locate the first sequence overlapping flat tile `start` (warp-cooperative).
-__device__ inline void locate_warp(const int32_t* seqlens, int B, int L_max, long long start, int* b_out,
+// Locate the first sequence overlapping flat unit `start` (warp-cooperative).
+__device__ inline void locate_warp(const int32_t* seqlens, int B, int L_max, int S, long long start, int* b_out,
                                    long long* acc_out) {
     const int lane = threadIdx.x & 31;
     long long acc = 0;
     for (int base = 0; base < B; base += 32) {
         const int b = base + lane;
-        const long long n = (b < B) ? num_tiles(clamp_len(seqlens[b], L_max, nullptr)) : 0;
+        const long long n = (b < B) ? num_units(clamp_len(seqlens[b], L_max, nullptr), S) : 0;
         // inclusive prefix within the warp
         long long incl = n;
 #pragma unroll
@@ -108,11 +125,14 @@ struct Piece {
 struct PieceWalker {
     const int32_t* seqlens;
     int B, L_max, p;
-    long long start, end;  // flat tile range of this partition
+    int S;                 // 0: balanced schedule over tiles; > 0: chunks of S tiles
+    long long start, end;  // flat unit range of this partition
     int b;                 // next sequence to look at
-    long long acc;         // its flat offset
+    long long acc;         // its flat offset (in units)
+    long long k;           // S > 0: next chunk of sequence b
 
     __device__ bool next(Piece& out) {
+        if (S > 0) return next_chunk(out);
         while (b < B && acc < end) {
             const int L = clamp_len(seqlens[b], L_max, nullptr);
             const long long n = num_tiles(L);
@@ -131,6 +151,30 @@ struct PieceWalker {
             const bool continues_after = acc_cur + n > end;
             if (!starts_before && !continues_after) out.slot = -1;
             else out.slot = starts_before ? 2 * p : 2 * p + 1;
+            return true;
+        }
+        return false;
+    }
+
+    // batch-invariant schedule: one S-tile chunk per piece
+    __device__ bool next_chunk(Piece& out) {
+        while (b < B && acc + k < end) {
+            const int L = clamp_len(seqlens[b], L_max, nullptr);
+            const long long n = num_tiles(L);
+            const long long u = (n + S - 1) / S;
+            if (acc + k < start) k = start - acc;
+            if (k >= u) {
+                acc += u;
+                ++b;
+                k = 0;
+                continue;
+            }
+            out.b = b;
+            out.L = L;
+            out.tile_lo = static_cast<int>(k * S);
+            out.tile_hi = static_cast<int>((k + 1) * S < n ? (k + 1) * S : n);
+            out.slot = (u == 1) ? -1 : static_cast<int>(acc + k);
+            ++k;
             return true;
         }
         return false;

@@ -108,3 +108,17 @@ def test_run_rejects_without_launching(lib):
 
 def test_check_rejects_null(lib):
     assert lib.mla_decode_check(None, None, None) == 1
+
+
+def test_batch_invariant_plan_without_gpu():
+    p = M.mla_decode_plan_batch_invariant(64, 1, 128, 8192, device=-1)
+    assert p.split_tiles == 16 and p.kernel == M.MLA_KERNEL_PAIR
+    # one fp32 partial (512 values + lse) per 16-tile chunk of every sequence at L_max
+    slots = 64 * (8192 // 128 // 16)
+    assert p.workspace_bytes >= slots * 128 * 513 * 4
+    q = M.mla_decode_plan_batch_invariant(64, 1, 16, 8192, device=-1, split_tiles=5)
+    assert q.split_tiles == 5 and q.kernel == M.MLA_KERNEL_TRANSPOSED
+    b = M.mla_decode_plan(64, 1, 128, 8192, device=-1)
+    assert b.split_tiles == 0
+    with pytest.raises(M.MlaError):
+        M.mla_decode_plan_batch_invariant(64, 1, 128, 8192, device=-1, split_tiles=-1)
