@@ -44,14 +44,23 @@ __global__ void __launch_bounds__(kCombineThreads)
     mla_decode_combine_kernel(const CombineArgs args) {
     __shared__ long long red_acc[kCombineThreads / 32];
     __shared__ long long red_tot[kCombineThreads / 32];
+    __shared__ int s_split;
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    // the schedule the main kernel used for these lengths
+    if (warp == 0) {
+        const int se = schedule_scan_warp(args.seqlens, args.B, args.L_max, args.P, args.split_tiles).S;
+        if (lane == 0) s_split = se;
+    }
+    __syncthreads();
+    const int S = s_split;
+
     // flat unit offset of sequence b, and the total (units: tiles, or S-tile chunks)
     long long acc = 0, tot = 0;
     for (int i = threadIdx.x; i < args.B; i += kCombineThreads) {
-        const long long n = num_units(clamp_len(args.seqlens[i], args.L_max, nullptr), args.split_tiles);
+        const long long n = num_units(clamp_len(__ldg(args.seqlens + i), args.L_max, nullptr), S);
         tot += n;
         if (i < b) acc += n;
     }
@@ -72,8 +81,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     const int r = blockIdx.y * kCombineRowsPerCta + warp;  // this warp's query row
     if (r >= args.R) return;
     const size_t orow = static_cast<size_t>(b) * args.R + r;
-    const int L = clamp_len(args.seqlens[b], args.L_max, nullptr);
-    const long long n = num_units(L, args.split_tiles);
+    const int L = clamp_len(__ldg(args.seqlens + b), args.L_max, nullptr);
+    const long long n = num_units(L, S);
     // a per-head sink is one more softmax term without a value (-inf: none)
     const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
     if (n == 0) {
@@ -84,8 +93,8 @@ __global__ void __launch_bounds__(kCombineThreads)
         return;
     }
     int k, p0 = 0;
-    if (args.split_tiles > 0) {
-        // batch-invariant chunks: chunk i of b is in slot acc + i
+    if (S > 0) {
+        // chunk schedule: chunk i of b is in slot acc + i
         if (n == 1) return;  // one chunk: finished by the main kernel
         k = static_cast<int>(n);
     } else {
@@ -98,7 +107,7 @@ __global__ void __launch_bounds__(kCombineThreads)
     // slot of the i-th piece: the first partition's piece continues after it
     // (2 p0 + 1), every later piece started before its partition (2 p)
     auto slot_of = [&](int i) {
-        if (args.split_tiles > 0) return static_cast<int>(acc) + i;
+        if (S > 0) return static_cast<int>(acc) + i;
         return (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i);
     };
 

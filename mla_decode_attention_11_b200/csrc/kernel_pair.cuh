@@ -118,6 +118,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     int* b_first_slot = reinterpret_cast<int*>(misc + 2);
     long long* acc_first_slot = reinterpret_cast<long long*>(misc + 4);
     long long* total_slot = reinterpret_cast<long long*>(misc + 6);
+    int* split_slot = reinterpret_cast<int*>(misc + 8);  // schedule chunk size of this run (0: balanced)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -159,15 +160,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         ptx::tmem_relinquish_pair();
     }
     if (warp == 0) {
-        const long long total = total_units_warp(args.seqlens, args.B, args.L_max, args.split_tiles);
+        const ScheduleScan sc = schedule_scan_warp(args.seqlens, args.B, args.L_max, args.P, args.split_tiles);
+        const int S_eff = sc.S;
+        const long long total = sc.units;
         const long long T = (total + args.P - 1) / args.P;
         int bf;
         long long af;
-        locate_warp(args.seqlens, args.B, args.L_max, args.split_tiles, static_cast<long long>(p) * T, &bf, &af);
+        locate_warp(args.seqlens, args.B, args.L_max, S_eff, static_cast<long long>(p) * T, &bf, &af);
         if (lane == 0) {
             *b_first_slot = bf;
             *acc_first_slot = af;
             *total_slot = total;
+            *split_slot = S_eff;
         }
         if (blockIdx.x == 0)
             for (int b = lane; b < args.B; b += 32) clamp_len(args.seqlens[b], args.L_max, args.status);
@@ -191,7 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         walker.B = args.B;
         walker.L_max = args.L_max;
         walker.p = p;
-        walker.S = args.split_tiles;
+        walker.S = *split_slot;
         walker.k = 0;
         walker.start = static_cast<long long>(p) * T;
         walker.end = walker.start + T < total ? walker.start + T : total;

@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(192, 1)
     int* b_first_slot = reinterpret_cast<int*>(misc + 2);
     long long* acc_first_slot = reinterpret_cast<long long*>(misc + 4);
     long long* total_slot = reinterpret_cast<long long*>(misc + 6);
+    int* split_slot = reinterpret_cast<int*>(misc + 8);  // schedule chunk size of this run (0: balanced)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -221,17 +222,20 @@ __global__ void __launch_bounds__(192, 1)
         ptx::tmem_relinquish();
     }
     if (warp == 0) {
+        const ScheduleScan sc = schedule_scan_warp(args.seqlens, args.B, args.L_max, args.P, args.split_tiles);
+        const int S_eff = sc.S;
         // partition bounds in the flat tile space, and the first sequence
-        const long long total = total_units_warp(args.seqlens, args.B, args.L_max, args.split_tiles);
+        const long long total = sc.units;
         const long long T = (total + args.P - 1) / args.P;
         const long long start = static_cast<long long>(p) * T;
         int bf;
         long long af;
-        locate_warp(args.seqlens, args.B, args.L_max, args.split_tiles, start, &bf, &af);
+        locate_warp(args.seqlens, args.B, args.L_max, S_eff, start, &bf, &af);
         if (lane == 0) {
             *b_first_slot = bf;
             *acc_first_slot = af;
             *total_slot = total;
+            *split_slot = S_eff;
         }
         // flag out-of-range lengths once (partition 0, group 0 only)
         if (blockIdx.x == 0)
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
         walker.B = args.B;
         walker.L_max = args.L_max;
         walker.p = p;
-        walker.S = args.split_tiles;
+        walker.S = *split_slot;
         walker.k = 0;
         walker.start = static_cast<long long>(p) * T;
         walker.end = walker.start + T < total ? walker.start + T : total;

@@ -73,11 +73,50 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
     return v;
 }
 
-__device__ inline long long total_units_warp(const int32_t* seqlens, int B, int L_max, int S) {
+// Schedule actually used for a run (warp-cooperative; every CTA and the
+// combine kernel reach the same answer from the same lengths).  A plan's
+// split_tiles > 0 (batch-invariant) is kept.  Otherwise the balanced schedule
+// is used, except when a whole sequence per partition is expected to finish
+// sooner: cutting a sequence costs about kCutTiles tiles of time (an extra
+// epilogue that stalls the pipeline, the fp32 partials and their merge), and
+// a balanced partition holds up to two cut pieces.  So when every non-empty
+// sequence fits its own partition, the sequences keep at least half of the
+// partitions busy, and the longest sequence is no longer than the balanced
+// share plus two cuts, each sequence is one piece (returned as a chunk size
+// covering the longest sequence).
+constexpr long long kCutTiles = 5;
+
+struct ScheduleScan {
+    int S;            // chunk size in tiles of this run's schedule (0: balanced over tiles)
+    long long units;  // schedule units over all sequences (tiles, or chunks)
+};
+
+// One pass over the lengths (warp-cooperative): the schedule of this run and
+// its number of units.
+__device__ inline ScheduleScan schedule_scan_warp(const int32_t* seqlens, int B, int L_max, int P, int plan_split) {
     const int lane = threadIdx.x & 31;
-    long long s = 0;
-    for (int b = lane; b < B; b += 32) s += num_units(clamp_len(seqlens[b], L_max, nullptr), S);
-    return warp_sum_ll(s);
+    long long total = 0, n_max = 0, nonempty = 0, chunks = 0;
+    for (int b = lane; b < B; b += 32) {
+        const int L = clamp_len(__ldg(seqlens + b), L_max, nullptr);
+        const long long n = num_tiles(L);
+        total += n;
+        n_max = n > n_max ? n : n_max;
+        nonempty += (n > 0);
+        if (plan_split > 0) chunks += num_units(L, plan_split);
+    }
+    total = warp_sum_ll(total);
+    nonempty = warp_sum_ll(nonempty);
+    chunks = warp_sum_ll(chunks);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const long long y = __shfl_xor_sync(0xffffffffu, n_max, o);
+        n_max = y > n_max ? y : n_max;
+    }
+    if (plan_split > 0) return {plan_split, chunks};
+    if (n_max == 0 || nonempty > P || 2 * nonempty < P) return {0, total};
+    const long long T = (total + P - 1) / P;
+    if (n_max <= T + 2 * kCutTiles) return {static_cast<int>(n_max), nonempty};
+    return {0, total};
 }
 
 // Locate the first sequence overlapping flat unit `start` (warp-cooperative).
@@ -87,7 +126,7 @@ __device__ inline void locate_warp(const int32_t* seqlens, int B, int L_max, int
     long long acc = 0;
     for (int base = 0; base < B; base += 32) {
         const int b = base + lane;
-        const long long n = (b < B) ? num_units(clamp_len(seqlens[b], L_max, nullptr), S) : 0;
+        const long long n = (b < B) ? num_units(clamp_len(__ldg(seqlens + b), L_max, nullptr), S) : 0;
         // inclusive prefix within the warp
         long long incl = n;
 #pragma unroll
@@ -134,7 +173,7 @@ struct PieceWalker {
     __device__ bool next(Piece& out) {
         if (S > 0) return next_chunk(out);
         while (b < B && acc < end) {
-            const int L = clamp_len(seqlens[b], L_max, nullptr);
+            const int L = clamp_len(__ldg(seqlens + b), L_max, nullptr);
             const long long n = num_tiles(L);
             const long long lo = acc > start ? acc : start;
             const long long hi = (acc + n) < end ? (acc + n) : end;
@@ -159,7 +198,7 @@ struct PieceWalker {
     // batch-invariant schedule: one S-tile chunk per piece
     __device__ bool next_chunk(Piece& out) {
         while (b < B && acc + k < end) {
-            const int L = clamp_len(seqlens[b], L_max, nullptr);
+            const int L = clamp_len(__ldg(seqlens + b), L_max, nullptr);
             const long long n = num_tiles(L);
             const long long u = (n + S - 1) / S;
             if (acc + k < start) k = start - acc;

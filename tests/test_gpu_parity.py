@@ -143,6 +143,15 @@ def test_rising_scores_force_rescale(cuda_device):
     assert_parity(out, lse, ro, rl, "ramp")
 
 
+@pytest.mark.parametrize("B,L,H", [(40, 300, 128), (30, 300, 128), (100, 700, 64), (150, 260, 16)])
+def test_uniform_batches_either_schedule(cuda_device, B, L, H):
+    """Equal lengths with enough sequences to fill at least half the
+    partitions switch the device schedule to one piece per sequence (no cuts);
+    fewer sequences keep the balanced split.  Both must match the oracle."""
+    w = W.custom(B=B, Sq=1, H=H, L=L, seed=600 + B)
+    check_workload(w)
+
+
 def test_split_matches_unsplit(cuda_device):
     w = W.custom(B=3, Sq=1, H=128, L=3000, seed=80)
     q, kv, sl = W.generate(w)
