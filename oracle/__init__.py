@@ -62,6 +62,9 @@ def _load():
             lib.oracle_mla_decode_rows_sinks.restype = ctypes.c_int
             lib.oracle_mla_decode_rows_sinks.argtypes = [ptr, ptr, ptr, i64, i64, i64, i64, i64, i64,
                                                          dbl, ptr, ptr, i64, ptr, ptr, ctypes.c_int]
+            lib.oracle_mha_decode.restype = ctypes.c_int
+            lib.oracle_mha_decode.argtypes = [ptr, ptr, ptr, ptr, i64, i64, i64, i64, i64, i64, i64,
+                                              dbl, ptr, ptr, ctypes.c_int]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -138,4 +141,29 @@ def mla_decode_rows(q, kv, seqlens, scale: float, row_ids, d_v: int = 512, num_t
                                               out.ctypes.data, lse.ctypes.data, int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle_mla_decode_rows failed with code {rc}")
+    return out, lse
+
+
+def mha_decode(q, k, v, seqlens, scale: float, num_threads: int = 0):
+    """MHA decode oracle: q [B,Sq,H,D], k [B,L_max,Hkv,D], v [B,L_max,Hkv,Dv]
+    (bf16), seqlens int [B]; head h reads kv head h // (H // Hkv).
+    Returns (out float64 [B,Sq,H,Dv], lse float64 [B,Sq,H])."""
+    qb, kb, vb = _as_bf16_bits(q), _as_bf16_bits(k), _as_bf16_bits(v)
+    if qb.ndim != 4 or kb.ndim != 4 or vb.ndim != 4:
+        raise ValueError("q must be [B,Sq,H,D], k [B,L_max,Hkv,D] and v [B,L_max,Hkv,Dv]")
+    B, Sq, H, D = qb.shape
+    _, L_max, Hkv, Dk = kb.shape
+    Dv = vb.shape[3]
+    if Dk != D or kb.shape[0] != B or vb.shape[:3] != kb.shape[:3]:
+        raise ValueError("q, k and v disagree on B, L_max, Hkv or D")
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
+    if sl.shape[0] != B:
+        raise ValueError("seqlens must have B entries")
+    out = np.empty((B, Sq, H, Dv), dtype=np.float64)
+    lse = np.empty((B, Sq, H), dtype=np.float64)
+    rc = _load().oracle_mha_decode(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, sl.ctypes.data,
+                                   B, Sq, H, Hkv, L_max, D, Dv, float(scale),
+                                   out.ctypes.data, lse.ctypes.data, int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_mha_decode failed with code {rc}")
     return out, lse

@@ -229,3 +229,93 @@ int oracle_max_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------
+ * MHA decode (the second workload on the same skeleton): standard
+ * multi-head attention with a separate V tensor and grouped KV heads.  The
+ * TileLang summary lists MHA in its main-results table (section "主实验",
+ * row "MHA", matched against FlashAttention-3) and uses it as the base the
+ * attention-sink variant differs from ("关键发现").  No formula is printed;
+ * this is the textbook definition:
+ *
+ *   for sequence b, token t < Sq, head h < H, kv head hk = h / (H / Hkv),
+ *   with L = seqlens[b]:
+ *     s_j          = scale * sum_{d < D} q[b,t,h,d] * k[b,j,hk,d]      (j < L)
+ *     out[b,t,h,e] = sum_j exp(s_j - m) * v[b,j,hk,e] / l              (e < Dv)
+ *     lse[b,t,h]   = m + ln(l),   m = max_j s_j,   l = sum_j exp(s_j - m)
+ *
+ * Same arithmetic rules as above (exact widening, index-order sums, two
+ * passes, no blocking); L = 0 gives out = 0, lse = -inf.
+ *   q : bf16 [B, Sq, H, D];  k : bf16 [B, L_max, Hkv, D];  v : bf16 [B, L_max, Hkv, Dv]
+ *   out : double [B, Sq, H, Dv];  lse : double [B, Sq, H]
+ * ------------------------------------------------------------------------ */
+static void mha_one_row(const uint16_t *q_row, const uint16_t *k_seq, const uint16_t *v_seq,
+                        int64_t L, int64_t Hkv, int64_t hk, int64_t D, int64_t Dv, double scale,
+                        double *scores, double *out_row, double *lse_out)
+{
+    if (L <= 0) {
+        for (int64_t e = 0; e < Dv; ++e) out_row[e] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    for (int64_t j = 0; j < L; ++j) {
+        const uint16_t *k_row = k_seq + (j * Hkv + hk) * D;
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d)
+            dot += bf16_bits_to_double(q_row[d]) * bf16_bits_to_double(k_row[d]);
+        scores[j] = scale * dot;
+    }
+    double m = scores[0];
+    for (int64_t j = 1; j < L; ++j)
+        if (scores[j] > m) m = scores[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+        scores[j] = exp(scores[j] - m);
+        l += scores[j];
+    }
+    for (int64_t e = 0; e < Dv; ++e) out_row[e] = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+        const uint16_t *v_row = v_seq + (j * Hkv + hk) * Dv;
+        const double w = scores[j];
+        for (int64_t e = 0; e < Dv; ++e)
+            out_row[e] += w * bf16_bits_to_double(v_row[e]);
+    }
+    for (int64_t e = 0; e < Dv; ++e) out_row[e] /= l;
+    *lse_out = m + log(l);
+}
+
+int oracle_mha_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *seqlens,
+                      int64_t B, int64_t Sq, int64_t H, int64_t Hkv, int64_t L_max, int64_t D, int64_t Dv,
+                      double scale, double *out, double *lse, int num_threads)
+{
+    if (!q || !k || !v || !seqlens || !out || !lse) return -1;
+    if (B < 0 || Sq < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || L_max < 0 || D < 1 || Dv < 1) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > L_max) return -1;
+    const int64_t rows = B * Sq * H;
+    const int64_t group = H / Hkv;
+    int failed = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(L_max > 0 ? L_max : 1));
+        if (!scores) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t r = 0; r < rows; ++r) {
+                const int64_t b = r / (Sq * H);
+                const int64_t h = r % H;
+                mha_one_row(q + r * D, k + b * L_max * Hkv * D, v + b * L_max * Hkv * Dv, seqlens[b], Hkv,
+                            h / group, D, Dv, scale, scores, out + r * Dv, lse + r);
+            }
+            free(scores);
+        }
+    }
+    return failed ? -2 : 0;
+}

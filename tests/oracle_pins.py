@@ -307,3 +307,78 @@ def pin_sink_empty_sequence(impl):
 
 SINK_PINS = [pin_sink_absent_is_minus_inf, pin_sink_zero_query, pin_sink_is_a_value_free_key,
              pin_sink_empty_sequence]
+
+
+# ---------------------------------------------------------------- MHA decode
+# impl(q, k, v, seqlens, scale) with q [B,Sq,H,D], k [B,L,Hkv,D], v [B,L,Hkv,Dv].
+
+def pin_mha_mqa_equals_latent_definition(impl):
+    """One kv head shared by all query heads, with v = the first Dv columns of
+    k, is exactly the latent-cache definition (keys are kv rows, values their
+    first Dv columns): compare with the MLA oracle's generic entry point."""
+    import oracle
+    g = torch.Generator().manual_seed(41)
+    q = _rand_bf16((2, 2, 4, 96), g)
+    k = _rand_bf16((2, 23, 1, 96), g)
+    v = k[..., :64].contiguous()
+    sl = np.array([23, 9], np.int32)
+    out, lse = impl(q, k, v, sl, 0.1)
+    ro, rl = oracle.mla_decode(q, k[:, :, 0, :].contiguous(), sl, 0.1, d_v=64)
+    np.testing.assert_allclose(out, ro, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-13)
+
+
+def pin_mha_sdpa_library(impl):
+    """torch's fp64 scaled_dot_product_attention with the kv heads repeated
+    over their query-head groups (GQA), and torch.logsumexp, at D = Dv = 128
+    with ragged lengths and two tokens."""
+    g = torch.Generator().manual_seed(42)
+    B, Sq, H, Hkv, L, D = 2, 2, 8, 2, 41, 128
+    q = _rand_bf16((B, Sq, H, D), g)
+    k = _rand_bf16((B, L, Hkv, D), g)
+    v = _rand_bf16((B, L, Hkv, D), g)
+    sl = np.array([41, 13], np.int32)
+    scale = D ** -0.5
+    out, lse = impl(q, k, v, sl, scale)
+    for b in range(B):
+        Lb = int(sl[b])
+        qq = q[b].double().permute(1, 0, 2)                                 # [H, Sq, D]
+        kk = k[b, :Lb].double().permute(1, 0, 2).repeat_interleave(H // Hkv, dim=0)  # [H, L, D]
+        vv = v[b, :Lb].double().permute(1, 0, 2).repeat_interleave(H // Hkv, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=scale)  # [H, Sq, D]
+        np.testing.assert_allclose(out[b], ref.permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+        sc = torch.einsum("hsd,hld->hsl", qq, kk) * scale
+        np.testing.assert_allclose(lse[b], torch.logsumexp(sc, dim=-1).permute(1, 0).numpy(), rtol=0, atol=1e-12)
+
+
+def pin_mha_head_groups(impl):
+    """Head h reads kv head h // (H / Hkv): with every value of kv head hk equal
+    to hk + 1, head h's output is exactly h // (H / Hkv) + 1 (the weights sum
+    to one), whatever the scores."""
+    g = torch.Generator().manual_seed(43)
+    B, H, Hkv, L, D = 1, 12, 3, 17, 64
+    q = _rand_bf16((B, 1, H, D), g, sigma=2.0)
+    k = _rand_bf16((B, L, Hkv, D), g, sigma=2.0)
+    v = torch.empty((B, L, Hkv, 32), dtype=torch.bfloat16)
+    for hk in range(Hkv):
+        v[:, :, hk, :] = hk + 1
+    out, _ = impl(q, k, v, np.array([L], np.int32), 0.2)
+    for h in range(H):
+        np.testing.assert_allclose(out[0, 0, h], h // (H // Hkv) + 1, rtol=1e-14, atol=0)
+
+
+def pin_mha_single_key(impl):
+    """L = 1: out is that key's value row of the head's kv head; lse its score."""
+    g = torch.Generator().manual_seed(44)
+    q = _rand_bf16((1, 1, 4, 128), g)
+    k = _rand_bf16((1, 3, 2, 128), g)
+    v = _rand_bf16((1, 3, 2, 128), g)
+    out, lse = impl(q, k, v, np.array([1], np.int32), 0.09)
+    for h in range(4):
+        hk = h // 2
+        np.testing.assert_array_equal(out[0, 0, h], _f64(v[0, 0, hk]))
+        s0 = 0.09 * float(torch.dot(q[0, 0, h].double(), k[0, 0, hk].double()))
+        assert abs(lse[0, 0, h] - s0) <= 1e-12 * max(1.0, abs(s0))
+
+
+MHA_PINS = [pin_mha_mqa_equals_latent_definition, pin_mha_sdpa_library, pin_mha_head_groups, pin_mha_single_key]

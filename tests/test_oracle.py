@@ -192,3 +192,64 @@ def test_pins_catch_planted_mistakes(name):
         assert failed == [], f"a correct stand-in must pass every pin, failed: {failed}"
     else:
         assert failed, f"planted mistake '{name}' passed every pin"
+
+
+
+# ---------------------------------------------------------------- MHA decode oracle
+
+def mha_oracle_impl(q, k, v, sl, scale):
+    return oracle.mha_decode(q, k, v, sl, scale)
+
+
+@pytest.mark.parametrize("pin", pins.MHA_PINS, ids=lambda p: p.__name__)
+def test_mha_oracle_pin(pin):
+    pin(mha_oracle_impl)
+
+
+def _np_mha(q, k, v, sl, scale, *, group_map="div", values_from_k=False, scale_used=True, len_delta=0):
+    qd, kd, vd = (x.to(torch.float64).numpy() for x in (q, k, v))
+    B, Sq, H, D = qd.shape
+    Hkv, Dv = kd.shape[2], vd.shape[3]
+    out = np.zeros((B, Sq, H, Dv))
+    lse = np.zeros((B, Sq, H))
+    for b in range(B):
+        L = max(0, min(int(sl[b]) + len_delta, kd.shape[1]))
+        for t in range(Sq):
+            for h in range(H):
+                hk = h // (H // Hkv) if group_map == "div" else h % Hkv
+                if L == 0:
+                    lse[b, t, h] = -np.inf
+                    continue
+                s = (kd[b, :L, hk] @ qd[b, t, h]) * (scale if scale_used else 1.0)
+                m = s.max()
+                w = np.exp(s - m)
+                vals = kd[b, :L, hk, :Dv] if values_from_k else vd[b, :L, hk]
+                out[b, t, h] = (w @ vals) / w.sum()
+                lse[b, t, h] = m + np.log(w.sum())
+    return out, lse
+
+
+MHA_MUTANTS = {
+    "correct": {},
+    "kv_head_h_mod_hkv": dict(group_map="mod"),
+    "values_from_k": dict(values_from_k=True),
+    "scale_ignored": dict(scale_used=False),
+    "one_key_short": dict(len_delta=-1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MHA_MUTANTS))
+def test_mha_pins_catch_planted_mistakes(name):
+    def impl(q, k, v, sl, scale):
+        return _np_mha(q, k, v, sl, scale, **MHA_MUTANTS[name])
+    failed = []
+    for pin in pins.MHA_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    if name == "correct":
+        assert failed == [], f"a correct stand-in must pass every MHA pin, failed: {failed}"
+    else:
+        assert failed, f"planted mistake '{name}' passed every MHA pin"
