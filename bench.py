@@ -365,13 +365,124 @@ def run_ours(args, w: W.Workload):
         dist.destroy_process_group()
 
 
+def run_mha(args, w: W.MhaWorkload):
+    """MHA decode (the second workload on the same skeleton): same timing
+    rules as run_ours, one GPU, no reference arm."""
+    from mla_decode_attention_11_b200 import binding as M
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    q, k, v, sl = W.generate_mha(w, tail_fill=0.0)
+    qd, kd, vd, sld = q.to(dev), k.to(dev), v.to(dev), sl.to(dev)
+    plan = M.mha_decode_plan(w.B, w.Sq, w.H, w.Hkv, w.L, device=0)
+    ws = M.alloc_workspace(plan, device=dev)
+    M.mla_decode_workspace_init(plan, ws)
+    out = torch.empty((w.B, w.Sq, w.H, W.MHA_D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def step():
+        M.mha_decode_run(plan, qd, kd, vd, sld, w.scale, out, lse, ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    M.mla_decode_check(plan, ws, stream=stream)
+
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    fn()
+        return g
+
+    def replay_ms(g, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / n
+
+    g_steps = capture(step, args.steps)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
+    t_ms = replay_ms(g_steps, args.steps)
+    clk = clocks.stop()
+    del g_steps
+    n_brk = max(3, min(args.steps, 50))
+    main_ms = replay_ms(capture(lambda: M.mha_decode_run_phase(plan, qd, kd, vd, sld, w.scale, out, lse, ws, 1,
+                                                               stream=stream), n_brk), n_brk)
+    comb_ms = replay_ms(capture(lambda: M.mha_decode_run_phase(plan, qd, kd, vd, sld, w.scale, out, lse, ws, 2,
+                                                               stream=stream), n_brk), n_brk)
+    M.mla_decode_check(plan, ws, stream=stream)
+    # end to end: host buffers in, host buffers out, copies inside the timed region
+    qh, kh, vh, slh = q.pin_memory(), k.pin_memory(), v.pin_memory(), sl.pin_memory()
+    outh = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            sld.copy_(slh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+            lseh.copy_(lse, non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    flops, nbytes = w.algorithmic_flops(sl), w.algorithmic_bytes(sl)
+    peaks, peak_src = load_peaks()
+    cpu_base = None
+    if not args.no_cpu_baseline:
+        import oracle
+        nb = min(w.B, 8)
+        t0 = time.perf_counter()
+        oracle.mha_decode(q[:nb], k[:nb], v[:nb], sl[:nb], w.scale)
+        dt = time.perf_counter() - t0
+        f_cpu = int(sl[:nb].to(torch.int64).sum()) * w.Sq * w.H * 2 * (2 * W.MHA_D)
+        cpu_base = {"value": f_cpu / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+                    "sample": f"{nb} of {w.B} sequences, all query rows, {dt:.1f} s of fp64 CPU work"}
+    achieved = nbytes / (main_ms * 1e-3) / 1e9
+    line = {
+        "metric": f"MHA decode TFLOP/s + HBM GB/s at B={w.B},H={w.H},Hkv={w.Hkv},d=128,L={w.L}; fraction of roofline",
+        "value": flops / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B={w.B} Sq={w.Sq} H={w.H} Hkv={w.Hkv} L={w.L}, d=128, bf16 "
+                               f"N(0,{w.sigma:g}) seed {w.seed}, scale 128^-0.5",
+                   "global_batch": w.B, "seq_len": w.L, "parallelism": "single GPU", "kernel": "transposed (MHA)",
+                   "group_rows": plan.group_rows, "partitions": plan.num_partitions,
+                   "l2": "inputs larger than L2, no flush"},
+        "hbm_gbs": nbytes / (t_ms * 1e-3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "kernel": "mla_decode_transposed_kernel<G, MhaShape>", "kernel_ms": main_ms,
+                     "combine_ms": comb_ms, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                     "step_roofline_frac": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3 / t_ms},
+        "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + sl.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 2 + lse.numel() * 4, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu_base,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="metric", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="metric", choices=sorted(W.WORKLOADS) + sorted(W.MHA_WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch-invariant", type=int, default=None, metavar="SPLIT_TILES",
                     help="use the batch-invariant plan, sequences cut every SPLIT_TILES KV tiles (0 = default)")
@@ -380,6 +491,12 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.workload in W.MHA_WORKLOADS:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the MLA workloads"}))
+            return
+        run_mha(args, W.MHA_WORKLOADS[args.workload])
+        return
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)

@@ -61,7 +61,8 @@ typedef enum mla_status {
 /* Kernel variants a plan can select. */
 enum {
     MLA_KERNEL_TRANSPOSED = 1, /* S^T = K Q^T per CTA, kv rows on the 128 TMEM lanes (any H*Sq) */
-    MLA_KERNEL_PAIR = 2        /* CTA pair, 64 query rows per CTA, cta_group::2 MMAs (H*Sq % 128 == 0) */
+    MLA_KERNEL_PAIR = 2,       /* CTA pair, 64 query rows per CTA, cta_group::2 MMAs (H*Sq % 128 == 0) */
+    MLA_KERNEL_MHA = 3         /* MHA decode (mha_decode_plan): the transposed kernel over 128-wide K, V */
 };
 
 /*
@@ -86,7 +87,10 @@ typedef struct mla_plan {
     int32_t split_tiles;       /* 0: balanced split-KV schedule (where a sequence is cut depends on the
                                   whole batch); > 0: batch-invariant schedule, every sequence cut into
                                   chunks of this many tiles (mla_decode_plan_batch_invariant) */
-    uint64_t reserved[5];
+    int32_t Hkv;               /* kv heads: 1 for MLA (one latent cache); MHA: query head h reads kv head
+                                  h / (H / Hkv) */
+    int32_t head_dim;          /* width of a key row: 576 (MLA), 128 (MHA) */
+    uint64_t reserved[4];
 } mla_plan;
 
 /*
@@ -271,6 +275,53 @@ mla_status mla_decode_check(const mla_plan* plan, void* workspace, void* stream)
 mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
                                   float softmax_scale, void* out, float* lse, int32_t wait_and_check,
                                   void* stream);
+
+/*
+ * MHA decode -- the second workload on the same skeleton: standard
+ * multi-head attention decode with grouped kv heads and separate K and V
+ * tensors of width 128.  The TileLang summary lists MHA in its main-results
+ * table ("TileLang: Bridging Programmability and Performance in Modern
+ * Neural Kernels", papernotes.org, section "主实验", row "MHA"); no formula
+ * is printed, and this is the textbook one.  For sequence b, token t, head h,
+ * kv head hk = h / (H / Hkv), L = seqlens[b]:
+ *     s_j = scale * <q[b,t,h,:], k[b,j,hk,:]>   (j < L)
+ *     out[b,t,h,:] = sum_j softmax(s)_j v[b,j,hk,:],   lse = ln sum_j exp(s_j)
+ * The Sq tokens of a sequence all see keys 0..L-1.  It runs on the transposed
+ * kernel: one CTA per (KV partition, kv head), its columns the Sq * (H / Hkv)
+ * query rows that share the kv head, padded to 16 or 32.
+ *
+ * mha_decode_plan -- as mla_decode_plan, with
+ *   H, Hkv     query and kv heads: 1 <= Hkv, H % Hkv == 0, Sq * (H / Hkv) <= 32
+ *   B, Sq, L_max, device, num_partitions_override, plan, workspace_bytes
+ *              as mla_decode_plan (Sq <= 16)
+ * Returns MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED or MLA_ERR_CUDA.
+ */
+mla_status mha_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t Hkv, int32_t L_max, int32_t device,
+                           int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
+
+/*
+ * mha_decode_run -- enqueue one MHA decode on `stream`.
+ *   q       device, bf16 [B, Sq, H, 128], contiguous, 16-byte aligned
+ *   k, v    device, bf16 [B, L_max, Hkv, 128] each, contiguous, 16-byte aligned
+ *   seqlens device, int32 [B], as for mla_decode_run
+ *   softmax_scale  multiplies q.k (128^-0.5 for standard attention)
+ *   sinks   device fp32 [H] per-head attention-sink logits (see
+ *           mla_decode_run_sinks) or NULL
+ *   out     device, bf16 [B, Sq, H, 128] (written);  lse  device, fp32 [B, Sq, H]
+ *   workspace  as for mla_decode_run, plan->workspace_bytes
+ * Launches the main kernel and the split-KV combine; no host sync, no
+ * allocation.  Return codes as mla_decode_run; MLA_ERR_INVALID_ARG for a
+ * plan not made by mha_decode_plan.
+ */
+mla_status mha_decode_run(const mla_plan* plan, const void* q, const void* k, const void* v, const int32_t* seqlens,
+                          float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/* mha_decode_run_phase -- the launches of mha_decode_run one at a time (1 =
+ * main kernel, 2 = split-KV combine), as mla_decode_run_phase. */
+mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void* k, const void* v,
+                                const int32_t* seqlens, float softmax_scale, const float* sinks, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream, int32_t phase);
 
 /* Static English description of a status code (never NULL). */
 const char* mla_status_string(mla_status status);

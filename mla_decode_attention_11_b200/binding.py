@@ -32,11 +32,14 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_ALIGNMENT", 3
                 4: "MLA_ERR_CUDA", 5: "MLA_ERR_TIMEOUT", 6: "MLA_ERR_WORKSPACE", 7: "MLA_ERR_SEQLEN"}
 MLA_KERNEL_TRANSPOSED = 1
 MLA_KERNEL_PAIR = 2
+MLA_KERNEL_MHA = 3
+MHA_D = 128
 MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
 EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_plan_batch_invariant", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
                     "mla_decode_check", "mla_decode_run_noalloc", "mla_decode_run_sinks",
-                    "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug")
+                    "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug",
+                    "mha_decode_plan", "mha_decode_run", "mha_decode_run_phase")
 
 
 class MlaError(RuntimeError):
@@ -52,7 +55,8 @@ class mla_plan(ctypes.Structure):
                 ("num_partitions", ctypes.c_int32), ("tile_kv", ctypes.c_int32), ("cta_threads", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_uint64), ("workspace_bytes", ctypes.c_uint64),
                 ("l2_prefetch_tiles", ctypes.c_int32), ("split_tiles", ctypes.c_int32),
-                ("reserved", ctypes.c_uint64 * 5)]
+                ("Hkv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("reserved", ctypes.c_uint64 * 4)]
 
     def as_dict(self):
         return {k: getattr(self, k) for k, _ in self._fields_ if not k.startswith("reserved")}
@@ -102,6 +106,15 @@ def load_library(build_if_missing: bool = True):
         lib.mla_decode_run_noalloc.restype = c_i32
         lib.mla_decode_run_noalloc.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_i32,
                                                c_vp]
+        lib.mha_decode_plan.restype = c_i32
+        lib.mha_decode_plan.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(mla_plan),
+                                        ctypes.POINTER(c_sz)]
+        lib.mha_decode_run.restype = c_i32
+        lib.mha_decode_run.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp, c_vp,
+                                       c_sz, c_vp]
+        lib.mha_decode_run_phase.restype = c_i32
+        lib.mha_decode_run_phase.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp,
+                                             c_vp, c_sz, c_vp, c_i32]
         lib.mla_decode_check.restype = c_i32
         lib.mla_decode_check.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp]
         lib.mla_status_string.restype = ctypes.c_char_p
@@ -322,3 +335,53 @@ def mla_decode_host(q_host: torch.Tensor, kv_host: torch.Tensor, seqlens_host: t
     out_host.copy_(dev_bufs["out"], non_blocking=True)
     lse_host.copy_(dev_bufs["lse"], non_blocking=True)
     return out_host, lse_host
+
+
+# ---------------------------------------------------------------- MHA decode
+
+def mha_decode_plan(B: int, Sq: int, H: int, Hkv: int, L_max: int, device: Optional[int] = None,
+                    num_partitions: int = 0) -> mla_plan:
+    """Plan an MHA decode (128-wide heads, H query heads over Hkv kv heads)."""
+    if device is None:
+        device = torch.cuda.current_device()
+    p = mla_plan()
+    ws = ctypes.c_size_t(0)
+    rc = load_library().mha_decode_plan(int(B), int(Sq), int(H), int(Hkv), int(L_max), int(device),
+                                        int(num_partitions), ctypes.byref(p), ctypes.byref(ws))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mha_decode_plan")
+    return p
+
+
+def mha_decode_run(plan: mla_plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seqlens: torch.Tensor,
+                   softmax_scale: float, out: torch.Tensor, lse: torch.Tensor, workspace: torch.Tensor,
+                   sinks: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Enqueue one MHA decode: q [B,Sq,H,128], k and v [B,L_max,Hkv,128] (bf16)."""
+    B, Sq, H, L, Hkv = plan.B, plan.Sq, plan.H, plan.L_max, plan.Hkv
+    _check_tensor(q, "q", torch.bfloat16, (B, Sq, H, MHA_D))
+    _check_tensor(k, "k", torch.bfloat16, (B, L, Hkv, MHA_D))
+    _check_tensor(v, "v", torch.bfloat16, (B, L, Hkv, MHA_D))
+    _check_tensor(seqlens, "seqlens", torch.int32, (B,))
+    _check_tensor(out, "out", torch.bfloat16, (B, Sq, H, MHA_D))
+    _check_tensor(lse, "lse", torch.float32, (B, Sq, H))
+    if sinks is not None:
+        _check_tensor(sinks, "sinks", torch.float32, (H,))
+    rc = load_library().mha_decode_run(ctypes.byref(plan), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                       seqlens.data_ptr(), float(softmax_scale),
+                                       sinks.data_ptr() if sinks is not None else None, out.data_ptr(),
+                                       lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                       _stream_handle(stream))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mha_decode_run")
+
+
+def mha_decode_run_phase(plan: mla_plan, q, k, v, seqlens, softmax_scale: float, out, lse, workspace, phase: int,
+                         sinks=None, stream=None) -> None:
+    """One launch of mha_decode_run (1 = main kernel, 2 = combine)."""
+    rc = load_library().mha_decode_run_phase(ctypes.byref(plan), q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                             seqlens.data_ptr(), float(softmax_scale),
+                                             sinks.data_ptr() if sinks is not None else None, out.data_ptr(),
+                                             lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                             _stream_handle(stream), int(phase))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mha_decode_run_phase")

@@ -40,8 +40,12 @@ struct CombineArgs {
 constexpr int kCombineThreads = 256;
 constexpr int kCombineRowsPerCta = kCombineThreads / 32;
 
+// DV: value width (512 for MLA, 128 for MHA); a lane owns DV / 128 float4 columns.
+template <int DV = kDv>
 __global__ void __launch_bounds__(kCombineThreads)
     mla_decode_combine_kernel(const CombineArgs args) {
+    static_assert(DV == 512 || DV == 128, "value width");
+    constexpr int NV4 = DV / 128;  // float4 columns per lane
     __shared__ long long red_acc[kCombineThreads / 32];
     __shared__ long long red_tot[kCombineThreads / 32];
     __shared__ int s_split;
@@ -86,9 +90,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     // a per-head sink is one more softmax term without a value (-inf: none)
     const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
     if (n == 0) {
-        uint4* dst = reinterpret_cast<uint4*>(args.out + orow * kDv);  // 64 x 16 bytes
-        dst[lane] = make_uint4(0u, 0u, 0u, 0u);
-        dst[lane + 32] = make_uint4(0u, 0u, 0u, 0u);
+        uint4* dst = reinterpret_cast<uint4*>(args.out + orow * DV);  // DV / 8 x 16 bytes
+        for (int i = lane; i < DV / 8; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
         if (lane == 0) args.lse[orow] = sink;  // nothing to attend to: the sink alone
         return;
     }
@@ -125,11 +128,11 @@ __global__ void __launch_bounds__(kCombineThreads)
     const float lse_all = m + logf(sum);
 
     // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
-    float4 acc_o[4];
+    float4 acc_o[NV4];
 #pragma unroll
-    for (int v = 0; v < 4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i0 = 0; i0 < k; i0 += 4) {
-        float4 x[4][4];
+        float4 x[4][NV4];
         float w[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -138,16 +141,16 @@ __global__ void __launch_bounds__(kCombineThreads)
             if (i < k) {
                 const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
                 w[j] = expf(args.part_lse[prow] - lse_all);
-                const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * kDv);
+                const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
 #pragma unroll
-                for (int v = 0; v < 4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
+                for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
             }
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             if (i0 + j < k) {
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
+                for (int v = 0; v < NV4; ++v) {
                     acc_o[v].x += w[j] * x[j][v].x;
                     acc_o[v].y += w[j] * x[j][v].y;
                     acc_o[v].z += w[j] * x[j][v].z;
@@ -156,9 +159,9 @@ __global__ void __launch_bounds__(kCombineThreads)
             }
         }
     }
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(args.out + orow * kDv);
+    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(args.out + orow * DV);
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
+    for (int v = 0; v < NV4; ++v) {
         const int e0 = (lane + 32 * v) * 4;  // first column of acc_o[v]
         const __nv_bfloat162 lo = __floats2bfloat162_rn(acc_o[v].x, acc_o[v].y);
         const __nv_bfloat162 hi = __floats2bfloat162_rn(acc_o[v].z, acc_o[v].w);

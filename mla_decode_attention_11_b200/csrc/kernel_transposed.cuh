@@ -60,6 +60,22 @@ struct MainArgs {
     const float* sinks;  // [H] per-head attention-sink logits (natural-log units), or null
     int H;               // heads: query row r of a sequence belongs to head r % H
     int split_tiles;     // 0: balanced schedule; > 0: batch-invariant chunks of this many tiles
+    int Sq;              // query tokens per sequence
+    int Hkv;             // MHA: kv heads (query head h reads kv head h / (H / Hkv)); MLA: 1
+};
+
+// The two attention shapes the transposed kernel serves.
+struct MlaShape {  // latent cache: keys are 576-wide kv rows, values their first 512 columns
+    static constexpr bool kMha = false;
+    static constexpr int kQKChunks = 9;  // 64-column chunks of a key (chunk 8 = rope)
+    static constexpr int kDvBlocks = 4;  // 128-wide blocks of a value row
+    static constexpr int kDv = 512;
+};
+struct MhaShape {  // multi-head attention: separate K and V tensors, 128 wide, grouped kv heads
+    static constexpr bool kMha = true;
+    static constexpr int kQKChunks = 2;
+    static constexpr int kDvBlocks = 1;
+    static constexpr int kDv = 128;
 };
 
 // Folds a per-head attention sink into a finished row.  (m, l) are the row's
@@ -78,12 +94,14 @@ __device__ __forceinline__ float fold_sink(float& m, float& l, float s2) {
 
 constexpr float kLog2e = 1.4426950408889634074f;
 
-template <int G>
+template <int G, class SH = MlaShape>
 struct TransposedCfg {
     static_assert(G == 16 || G == 32, "query rows per CTA");
     static constexpr int kThreads = 192;
-    static constexpr int NP = (G == 16) ? 5 : 4;  // pair slots (a tile needs 4)
-    static constexpr int NR = 2;                  // rope slots
+    // pair slots [128 kv x 128 col]: an MLA tile needs 4 (+ a rope slot), an MHA
+    // tile 2 (its K and its V)
+    static constexpr int NP = SH::kMha ? 6 : ((G == 16) ? 5 : 4);
+    static constexpr int NR = SH::kMha ? 1 : 2;   // rope slots (unused by MHA)
     static constexpr int kPairBytes = kTileKV * 128 * 2;     // 32 KB
     static constexpr int kChunkBytes = kTileKV * 128;        // 16 KB
     static constexpr int kQChunkBytes = G * 128;
@@ -91,7 +109,7 @@ struct TransposedCfg {
     static constexpr int OFF_PAIR = 0;
     static constexpr int OFF_ROPE = OFF_PAIR + NP * kPairBytes;
     static constexpr int OFF_Q = OFF_ROPE + NR * kChunkBytes;
-    static constexpr int OFF_PT = OFF_Q + kNumChunks * kQChunkBytes;
+    static constexpr int OFF_PT = OFF_Q + SH::kQKChunks * kQChunkBytes;
     static constexpr int OFF_RED = OFF_PT + kPTBytes;              // floats: [2][4][G] max, [4][G] sums
     static constexpr int kRedFloats = 12 * G;
     static constexpr int OFF_BAR = OFF_RED + kRedFloats * 4;
@@ -100,9 +118,11 @@ struct TransposedCfg {
     static constexpr int kNumBars = 7 + 2 * NP + 2 * NR;
     static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
     static constexpr int kSmemBytes = OFF_MISC + 64 + 1024;  // + slack to align the base to 1024
-    // TMEM: O^T blocks at columns [0, 4G), S^T at [4G, 5G)
-    static constexpr uint32_t kTmemCols = (5 * G <= 128) ? 128 : 256;
-    static constexpr uint32_t kColS = 4 * G;
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    // TMEM: O^T blocks at columns [0, kDvBlocks G), S^T after them
+    static constexpr int kCols = (SH::kDvBlocks + 1) * G;
+    static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : kCols <= 64 ? 64 : kCols <= 128 ? 128 : 256;
+    static constexpr uint32_t kColS = SH::kDvBlocks * G;
     // P^T swizzle: one row of G bf16 = 2G bytes (32 or 64)
     static constexpr ptx::Swizzle kPTSwz = (G == 16) ? ptx::Swizzle::B32 : ptx::Swizzle::B64;
     static constexpr uint32_t kPTAtom = 8 * 2 * G;  // 8 rows x row bytes
@@ -159,11 +179,23 @@ __device__ __forceinline__ int col_of_lane(int lane) {
     return (G == 32) ? lane : (lane >> 1);
 }
 
-template <int G>
+// MHA (SH = MhaShape): CTA group g is kv head g; its columns j < Sq * (H / Hkv)
+// are the query rows (token j / gq, head g gq + j % gq), gq = H / Hkv; the
+// remaining columns up to G are padding (zero Q, never stored).  tm_kv is K
+// and tm_v is V, both [B, L_max, Hkv, 128].  MLA: group g is query rows
+// [g G, g G + G) of the sequence and tm_v is unused.
+template <class SH>
+__device__ __forceinline__ int group_row(const MainArgs& a, int G, int g, int j) {
+    if (!SH::kMha) return g * G + j;
+    const int gq = a.H / a.Hkv;
+    return (j / gq) * a.H + g * gq + (j % gq);
+}
+
+template <int G, class SH = MlaShape>
 __global__ void __launch_bounds__(192, 1)
     mla_decode_transposed_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                                 const MainArgs args) {
-    using C = TransposedCfg<G>;
+                                 const __grid_constant__ CUtensorMap tm_v, const MainArgs args) {
+    using C = TransposedCfg<G, SH>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -244,6 +276,13 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 4 && lane == 0) {
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_kv);
+        if (SH::kMha) ptx::prefetch_tmap(&tm_v);
+    }
+    if (SH::kMha) {
+        // the Q rows past Sq * gq are padding that TMA never writes: make them zero
+        for (int i = threadIdx.x; i < SH::kQKChunks * C::kQChunkBytes / 16; i += C::kThreads)
+            reinterpret_cast<uint4*>(q_smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+        ptx::fence_proxy_async_smem();
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -279,15 +318,42 @@ __global__ void __launch_bounds__(192, 1)
                 // Q rows of this group: flattened [B*R, 576] rows b*R + g*G ...
                 if (piece_cnt > 0) ok = ptx::mbar_wait_bounded(q_empty, (piece_cnt - 1) & 1, tmo);
                 if (!ok) break;
-                ptx::mbar_arrive_expect_tx(q_full, kNumChunks * C::kQChunkBytes);
-                const int qrow = pc.b * args.R + g * G;
-                if (!(blockIdx.x == 0 && unit == args.stall_unit))
-                    for (int c = 0; c < kNumChunks; ++c)
-                        ptx::tma_load_2d(q_smem + c * C::kQChunkBytes, &tm_q, q_full, c * kChunk, qrow);
+                if (SH::kMha) {
+                    // q viewed as [B][Sq][H][128]: heads g gq .. g gq + gq - 1 of every token
+                    const int gq = args.H / args.Hkv;
+                    ptx::mbar_arrive_expect_tx(q_full, SH::kQKChunks * args.Sq * gq * 128);
+                    if (!(blockIdx.x == 0 && unit == args.stall_unit))
+                        for (int c = 0; c < SH::kQKChunks; ++c)
+                            ptx::tma_load_4d(q_smem + c * C::kQChunkBytes, &tm_q, q_full, c * kChunk, g * gq, 0, pc.b);
+                } else {
+                    ptx::mbar_arrive_expect_tx(q_full, kNumChunks * C::kQChunkBytes);
+                    const int qrow = pc.b * args.R + g * G;
+                    if (!(blockIdx.x == 0 && unit == args.stall_unit))
+                        for (int c = 0; c < kNumChunks; ++c)
+                            ptx::tma_load_2d(q_smem + c * C::kQChunkBytes, &tm_q, q_full, c * kChunk, qrow);
+                }
                 ++unit;
                 for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
                     int row0 = t * kTileKV;
                     if (row0 + kTileKV > pc.L) row0 = pc.L - kTileKV;  // end-aligned last tile
+                    if (SH::kMha) {
+                        // two pair slots: the tile's K rows, then its V rows (kv head g)
+                        for (int pp = 0; pp < 2; ++pp) {
+                            const uint32_t s = pair_cnt % C::NP;
+                            ok = ptx::mbar_wait_bounded(pair_empty + s, ((pair_cnt / C::NP) & 1) ^ 1, tmo);
+                            if (!ok) break;
+                            ptx::mbar_arrive_expect_tx(pair_full + s, C::kPairBytes);
+                            if (!(blockIdx.x == 0 && unit == args.stall_unit)) {
+                                uint8_t* dst = pair_smem + s * C::kPairBytes;
+                                const CUtensorMap* tm = (pp == 0) ? &tm_kv : &tm_v;
+                                ptx::tma_load_4d(dst, tm, pair_full + s, 0, g, row0, pc.b);
+                                ptx::tma_load_4d(dst + C::kChunkBytes, tm, pair_full + s, kChunk, g, row0, pc.b);
+                            }
+                            ++unit;
+                            ++pair_cnt;
+                        }
+                        continue;
+                    }
                     {
                         const uint32_t s = rope_cnt % C::NR;
                         ok = ptx::mbar_wait_bounded(rope_empty + s, ((rope_cnt / C::NR) & 1) ^ 1, tmo);
@@ -352,6 +418,50 @@ __global__ void __launch_bounds__(192, 1)
                     if (first) {
                         ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
                         if (!ok) break;
+                    }
+                    if (SH::kMha) {
+                        // ---------------- S^T = K . Q^T over the K pair, O^T += V^T . P^T over the V pair
+                        const uint32_t ks = pair_cnt % C::NP, vs = (pair_cnt + 1) % C::NP;
+                        ok = ptx::mbar_wait_bounded(pair_full + ks, (pair_cnt / C::NP) & 1, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        {
+                            const uint32_t kbase = ptx::smem_u32(pair_smem + ks * C::kPairBytes);
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk) {
+                                    const uint64_t da = ptx::make_smem_desc(kbase + h * C::kChunkBytes + kk * 32, 16,
+                                                                            1024, ptx::Swizzle::B128);
+                                    const uint64_t db = ptx::make_smem_desc(q_base + h * C::kQChunkBytes + kk * 32, 16,
+                                                                            1024, ptx::Swizzle::B128);
+                                    ptx::mma_bf16_ss(tm_S, da, db, C::kIdescS, (h | kk) ? 1u : 0u);
+                                }
+                            }
+                        }
+                        ptx::mma_commit(pair_empty + ks);
+                        if (last) ptx::mma_commit(q_empty);
+                        ptx::mma_commit(s_full);
+                        ok = ptx::mbar_wait_bounded(p_full, tile_cnt & 1, tmo) &&
+                             ptx::mbar_wait_bounded(pair_full + vs, ((pair_cnt + 1) / C::NP) & 1, tmo);
+                        if (!ok) break;
+                        ptx::tc_fence_after();
+                        {
+                            const uint32_t vbase = ptx::smem_u32(pair_smem + vs * C::kPairBytes);
+#pragma unroll
+                            for (int kk = 0; kk < kTileKV / 16; ++kk) {
+                                const uint64_t da =
+                                    ptx::make_smem_desc(vbase + kk * 2048, C::kChunkBytes, 1024, ptx::Swizzle::B128);
+                                const uint64_t db = ptx::make_smem_desc(pt_base + kk * 2 * C::kPTAtom, C::kPTBytes,
+                                                                        C::kPTAtom, C::kPTSwz);
+                                ptx::mma_bf16_ss(tmem_base, da, db, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                        ptx::mma_commit(pair_empty + vs);
+                        pair_cnt += 2;
+                        if (last) ptx::mma_commit(pv_done);
+                        ++tile_cnt;
+                        continue;
                     }
                     // ---------------- S^T = K . Q^T  (rope chunk first, then the 8 value chunks)
                     const uint32_t rs = rope_cnt % C::NR;
@@ -513,7 +623,7 @@ __global__ void __launch_bounds__(192, 1)
                     // O^T columns j *= alpha[j]; PV of the previous tile has
                     // completed (it was committed before this tile's S^T).
 #pragma unroll
-                    for (int blk = 0; blk < 4; ++blk) {
+                    for (int blk = 0; blk < SH::kDvBlocks; ++blk) {
 #pragma unroll
                         for (int c0 = 0; c0 < G; c0 += 16) {
                             uint32_t r[16];
@@ -560,32 +670,34 @@ __global__ void __launch_bounds__(192, 1)
             }
             ok = group_barrier();
             if (!ok) break;
-            const int row_base = g * G;  // first query row of this group within the sequence
+            // MHA: columns past Sq * gq are padding
+            const int n_cols = SH::kMha ? args.Sq * (args.H / args.Hkv) : G;
             // a sink applies once per row: to whole sequences here, to cut ones in the combine
             const bool sink_here = (args.sinks != nullptr) && (pc.slot < 0);
             // thread j < G finishes query row j (sum, sink, lse) and leaves its
             // 1 / l in the max buffer the piece's last tile did not use
             float* fin = red + (tile_cnt & 1) * 4 * G;
-            if (row_in_tile < G) {
+            if (row_in_tile < n_cols) {
                 const int j = row_in_tile;
+                const int qr = group_row<SH>(args, G, g, j);  // query row within the sequence
                 float mj = 0.f;
 #pragma unroll
                 for (int jj = 0; jj < G; ++jj)
                     if (jj == j) mj = m_ref[jj];
                 float lj = redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j];
                 float c = 1.f;
-                if (sink_here) c = fold_sink(mj, lj, args.sinks[(row_base + j) % args.H] * kLog2e);
+                if (sink_here) c = fold_sink(mj, lj, args.sinks[qr % args.H] * kLog2e);
                 fin[j] = c / lj;
                 const float lse_nat = (mj + log2f(lj)) * 0.69314718055994530942f;
                 if (pc.slot < 0)
-                    args.lse[static_cast<size_t>(pc.b) * args.R + row_base + j] = lse_nat;
+                    args.lse[static_cast<size_t>(pc.b) * args.R + qr] = lse_nat;
                 else
-                    args.part_lse[static_cast<size_t>(pc.slot) * args.R + row_base + j] = lse_nat;
+                    args.part_lse[static_cast<size_t>(pc.slot) * args.R + qr] = lse_nat;
             }
             ok = group_barrier();
             if (!ok) break;
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk) {
+            for (int blk = 0; blk < SH::kDvBlocks; ++blk) {
                 const int dv = blk * 128 + row_in_tile;
 #pragma unroll
                 for (int c0 = 0; c0 < G; c0 += 16) {
@@ -595,14 +707,17 @@ __global__ void __launch_bounds__(192, 1)
                     if (pc.slot < 0) {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const size_t orow = static_cast<size_t>(pc.b) * args.R + row_base + c0 + j;
-                            args.out[orow * kDv + dv] = __float2bfloat16_rn(__uint_as_float(r[j]) * fin[c0 + j]);
+                            if (c0 + j >= n_cols) continue;
+                            const size_t orow = static_cast<size_t>(pc.b) * args.R + group_row<SH>(args, G, g, c0 + j);
+                            args.out[orow * SH::kDv + dv] = __float2bfloat16_rn(__uint_as_float(r[j]) * fin[c0 + j]);
                         }
                     } else {
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
-                            const size_t orow = static_cast<size_t>(pc.slot) * args.R + row_base + c0 + j;
-                            args.part_o[orow * kDv + dv] = __uint_as_float(r[j]) * fin[c0 + j];
+                            if (c0 + j >= n_cols) continue;
+                            const size_t orow =
+                                static_cast<size_t>(pc.slot) * args.R + group_row<SH>(args, G, g, c0 + j);
+                            args.part_o[orow * SH::kDv + dv] = __uint_as_float(r[j]) * fin[c0 + j];
                         }
                     }
                 }

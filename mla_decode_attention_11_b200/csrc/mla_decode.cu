@@ -64,23 +64,23 @@ long long num_slots(const mla_plan& pl) {
     return 2LL * pl.num_partitions;
 }
 
-Layout workspace_layout(long long slots, int R) {
+Layout workspace_layout(long long slots, int R, int dv = mla::kDv) {
     Layout l;
     l.part_lse_off = kHeaderBytes;
     l.part_o_off = align_up(l.part_lse_off + size_t(slots) * R * sizeof(float), 256);
-    l.total = l.part_o_off + size_t(slots) * R * mla::kDv * sizeof(float);
+    l.total = l.part_o_off + size_t(slots) * R * dv * sizeof(float);
     return l;
 }
 
-template <int G>
+template <int G, class SH = mla::MlaShape>
 mla_status launch_transposed(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_kv,
-                             const mla::MainArgs& args, cudaStream_t stream) {
-    using C = mla::TransposedCfg<G>;
-    auto kern = mla::mla_decode_transposed_kernel<G>;
+                             const CUtensorMap& tm_v, const mla::MainArgs& args, cudaStream_t stream) {
+    using C = mla::TransposedCfg<G, SH>;
+    auto kern = mla::mla_decode_transposed_kernel<G, SH>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
         return MLA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(plan.num_partitions * plan.num_groups));
-    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, args);
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_v, args);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -219,6 +219,8 @@ mla_status mla_decode_plan_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_ma
     p.tile_kv = mla::kTileKV;
     p.l2_prefetch_tiles = kDefaultPrefetchTiles;
     p.split_tiles = 0;
+    p.Hkv = 1;
+    p.head_dim = mla::kDqk;
     p.workspace_bytes = workspace_layout(num_slots(p), R).total;
     *plan = p;
     if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
@@ -272,7 +274,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     } else if (pl.kernel == MLA_KERNEL_PAIR) {
         if (pl.group_rows != 128) return MLA_ERR_INVALID_ARG;
     } else {
-        return MLA_ERR_INVALID_ARG;
+        return MLA_ERR_INVALID_ARG;  // MHA plans run through mha_decode_run
     }
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
         !aligned(sinks, 4))
@@ -332,14 +334,16 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     a.sinks = sinks;
     a.H = pl.H;
     a.split_tiles = pl.split_tiles;
+    a.Sq = pl.Sq;
+    a.Hkv = 1;
 
     if (phases & 1) {
         mla_status st;
         if (pl.kernel == MLA_KERNEL_PAIR)
             st = launch_pair(pl, tm_q, tm_k, tm_kv, a, stream);
         else
-            st = (G == 16) ? launch_transposed<16>(pl, tm_q, tm_kv, a, stream)
-                           : launch_transposed<32>(pl, tm_q, tm_kv, a, stream);
+            st = (G == 16) ? launch_transposed<16>(pl, tm_q, tm_kv, tm_kv, a, stream)
+                           : launch_transposed<32>(pl, tm_q, tm_kv, tm_kv, a, stream);
         if (st != MLA_OK) {
             cudaGetLastError();
             return st;
@@ -361,7 +365,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     c.split_tiles = pl.split_tiles;
     const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) /
                                                                         mla::kCombineRowsPerCta));
-    mla::mla_decode_combine_kernel<<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
+    mla::mla_decode_combine_kernel<mla::kDv><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
 }
@@ -495,6 +499,204 @@ mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const voi
     if (word & mla::kStatusTimeout) return MLA_ERR_TIMEOUT;
     if (word & mla::kStatusSeqlen) return MLA_ERR_SEQLEN;
     return MLA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// MHA decode on the transposed kernel (MhaShape): q [B, Sq, H, 128], k and v
+// [B, L_max, Hkv, 128]; one CTA per (partition, kv head).
+// ---------------------------------------------------------------------------
+
+namespace {
+
+// a 4-D bf16 tensor, innermost dimension d[0] contiguous
+bool encode_4d_bf16(EncodeTiledFn enc, CUtensorMap* m, const void* base, const uint64_t d[4], const uint32_t box[4]) {
+    const cuuint64_t dims[4] = {d[0], d[1], d[2], d[3]};
+    const cuuint64_t strides[3] = {d[0] * 2, d[0] * d[1] * 2, d[0] * d[1] * d[2] * 2};
+    const cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, bx, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kMhaD = mla::MhaShape::kDv;  // 128: key and value width
+
+}  // namespace
+
+extern "C" {
+
+mla_status mha_decode_plan(int32_t B, int32_t Sq, int32_t H, int32_t Hkv, int32_t L_max, int32_t device,
+                           int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes) {
+    if (!plan) return MLA_ERR_INVALID_ARG;
+    if (B < 1 || B > 65535 || Sq < 1 || Sq > 16 || L_max < 1 || L_max > (1 << 24) || H < 1 || Hkv < 1 ||
+        H > 65535 || num_partitions_override < 0)
+        return MLA_ERR_INVALID_ARG;
+    if (H % Hkv != 0) return MLA_ERR_INVALID_ARG;
+    const int gq = H / Hkv;
+    if (Sq * gq > 32) return MLA_ERR_UNSUPPORTED;
+    int sms = 148;
+    if (device >= 0) {
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+            cudaGetLastError();
+            return MLA_ERR_CUDA;
+        }
+    }
+    mla_plan p;
+    std::memset(&p, 0, sizeof p);
+    p.B = B;
+    p.Sq = Sq;
+    p.H = H;
+    p.L_max = L_max;
+    p.device = device;
+    p.num_sms = sms;
+    p.kernel = MLA_KERNEL_MHA;
+    p.group_rows = (Sq * gq <= 16) ? 16 : 32;
+    p.num_groups = Hkv;
+    p.cta_threads = 192;
+    p.smem_bytes = (p.group_rows == 16) ? mla::TransposedCfg<16, mla::MhaShape>::kSmemBytes
+                                        : mla::TransposedCfg<32, mla::MhaShape>::kSmemBytes;
+    int P = num_partitions_override > 0 ? num_partitions_override : sms / Hkv;
+    if (P < 1) P = 1;
+    if (P > 4096) P = 4096;
+    p.num_partitions = P;
+    p.tile_kv = mla::kTileKV;
+    p.l2_prefetch_tiles = 0;
+    p.split_tiles = 0;
+    p.Hkv = Hkv;
+    p.head_dim = kMhaD;
+    p.workspace_bytes = workspace_layout(num_slots(p), Sq * H, kMhaD).total;
+    *plan = p;
+    if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
+    return MLA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+mla_status mha_run_phases(const mla_plan* plan, const void* q, const void* k, const void* v, const int32_t* seqlens,
+                          float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream_, int phases) {
+    if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
+    if (!plan || !q || !k || !v || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    const mla_plan& pl = *plan;
+    if (pl.kernel != MLA_KERNEL_MHA || pl.Hkv < 1 || pl.H < 1 || pl.H % pl.Hkv != 0 || pl.B < 1 || pl.Sq < 1 ||
+        pl.L_max < 1 || pl.num_partitions < 1 || pl.num_groups != pl.Hkv || pl.head_dim != kMhaD ||
+        pl.split_tiles < 0 || pl.split_tiles > (1 << 17))
+        return MLA_ERR_INVALID_ARG;
+    const int gq = pl.H / pl.Hkv;
+    const int G = pl.group_rows;
+    if ((G != 16 && G != 32) || pl.Sq * gq > G) return MLA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(seqlens, 4) || !aligned(sinks, 4))
+        return MLA_ERR_ALIGNMENT;
+    const int R = pl.Sq * pl.H;
+    const Layout lay = workspace_layout(num_slots(pl), R, kMhaD);
+    if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (pl.device >= 0 && dev != pl.device) return MLA_ERR_INVALID_ARG;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return MLA_ERR_CUDA;
+
+    CUtensorMap tm_q, tm_k, tm_v;
+    {
+        const uint64_t dq[4] = {static_cast<uint64_t>(kMhaD), static_cast<uint64_t>(pl.H),
+                                static_cast<uint64_t>(pl.Sq), static_cast<uint64_t>(pl.B)};
+        const uint32_t bq[4] = {static_cast<uint32_t>(mla::kChunk), static_cast<uint32_t>(gq),
+                                static_cast<uint32_t>(pl.Sq), 1u};
+        const uint64_t dk[4] = {static_cast<uint64_t>(kMhaD), static_cast<uint64_t>(pl.Hkv),
+                                static_cast<uint64_t>(pl.L_max), static_cast<uint64_t>(pl.B)};
+        const uint32_t bk[4] = {static_cast<uint32_t>(mla::kChunk), 1u, static_cast<uint32_t>(mla::kTileKV), 1u};
+        if (!encode_4d_bf16(enc, &tm_q, q, dq, bq) || !encode_4d_bf16(enc, &tm_k, k, dk, bk) ||
+            !encode_4d_bf16(enc, &tm_v, v, dk, bk))
+            return MLA_ERR_CUDA;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    mla::MainArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.seqlens = seqlens;
+    a.B = pl.B;
+    a.R = R;
+    a.L_max = pl.L_max;
+    a.P = pl.num_partitions;
+    a.NG = pl.num_groups;
+    a.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
+    a.part_lse = reinterpret_cast<float*>(ws + lay.part_lse_off);
+    a.status = reinterpret_cast<uint32_t*>(ws);
+    const unsigned long long tmo = g_timeout_ns.load();
+    a.timeout_ns = tmo ? tmo : kDefaultTimeoutNs;
+    a.stall_unit = g_stall_unit.load();
+    a.prefetch_tiles = 0;
+    a.sinks = sinks;
+    a.H = pl.H;
+    a.split_tiles = pl.split_tiles;
+    a.Sq = pl.Sq;
+    a.Hkv = pl.Hkv;
+    if (phases & 1) {
+        const mla_status st = (G == 16) ? launch_transposed<16, mla::MhaShape>(pl, tm_q, tm_k, tm_v, a, stream)
+                                        : launch_transposed<32, mla::MhaShape>(pl, tm_q, tm_k, tm_v, a, stream);
+        if (st != MLA_OK) {
+            cudaGetLastError();
+            return st;
+        }
+    }
+    if (!(phases & 2)) return MLA_OK;
+    mla::CombineArgs c;
+    std::memset(&c, 0, sizeof c);
+    c.seqlens = seqlens;
+    c.B = pl.B;
+    c.R = R;
+    c.L_max = pl.L_max;
+    c.P = pl.num_partitions;
+    c.out = a.out;
+    c.lse = lse;
+    c.part_o = a.part_o;
+    c.part_lse = a.part_lse;
+    c.sinks = sinks;
+    c.H = pl.H;
+    c.split_tiles = pl.split_tiles;
+    const dim3 cgrid(static_cast<unsigned>(pl.B),
+                     static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) / mla::kCombineRowsPerCta));
+    mla::mla_decode_combine_kernel<kMhaD><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    return MLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mla_status mha_decode_run(const mla_plan* plan, const void* q, const void* k, const void* v, const int32_t* seqlens,
+                          float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+    return mha_run_phases(plan, q, k, v, seqlens, softmax_scale, sinks, out, lse, workspace, workspace_bytes, stream,
+                          3);
+}
+
+mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void* k, const void* v,
+                                const int32_t* seqlens, float softmax_scale, const float* sinks, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream, int32_t phase) {
+    if (phase != 1 && phase != 2) return MLA_ERR_INVALID_ARG;
+    return mha_run_phases(plan, q, k, v, seqlens, softmax_scale, sinks, out, lse, workspace, workspace_bytes, stream,
+                          phase);
 }
 
 }  // extern "C"

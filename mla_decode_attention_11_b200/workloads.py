@@ -121,5 +121,76 @@ def ceil_div(a: int, b: int) -> int:
     return -(-a // b)
 
 
+# ---------------------------------------------------------------- MHA decode
+# Standard multi-head attention decode with grouped kv heads (128-wide heads,
+# separate K and V).  Same recipe: per sequence b, q[b] = randn(Sq, H, 128),
+# k[b, :L_b] = randn(L_b, Hkv, 128) and v[b, :L_b] = randn(L_b, Hkv, 128),
+# each from its own seeded generator, times sigma, rounded to bf16; rows past
+# L_b filled with tail_fill.
+
+MHA_D = 128
+
+
+@dataclasses.dataclass(frozen=True)
+class MhaWorkload:
+    name: str
+    B: int
+    Sq: int
+    H: int
+    Hkv: int
+    L: int
+    L_lo: Optional[int] = None
+    sigma: float = 1.0
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return float(torch.tensor(MHA_D ** -0.5, dtype=torch.float32).item())
+
+    def lengths(self) -> torch.Tensor:
+        return Workload(self.name, self.B, self.Sq, self.H, self.L, self.L_lo, self.sigma, self.seed).lengths()
+
+    def algorithmic_bytes(self, lengths: Optional[torch.Tensor] = None) -> int:
+        """Each used K and V row once (per kv head), q, out, lse, lengths."""
+        sl = self.lengths() if lengths is None else lengths
+        rows = self.B * self.Sq * self.H
+        return (int(sl.to(torch.int64).sum()) * self.Hkv * MHA_D * 2 * 2 + rows * (MHA_D * 2 * 2 + 4)
+                + self.B * 4)
+
+    def algorithmic_flops(self, lengths: Optional[torch.Tensor] = None) -> int:
+        """2*(128+128) flops per (query row, key)."""
+        sl = self.lengths() if lengths is None else lengths
+        return int(sl.to(torch.int64).sum()) * self.Sq * self.H * 2 * (2 * MHA_D)
+
+
+# a grouped-query decode batch (32 query heads over 8 kv heads of 128, 64
+# sequences of 8192 keys) and a small mixed-length case
+MHA_WORKLOADS = {
+    "mha_gqa": MhaWorkload("mha_gqa", B=64, Sq=1, H=32, Hkv=8, L=8192, seed=2001),
+    "mha_small": MhaWorkload("mha_small", B=6, Sq=2, H=16, Hkv=4, L=1500, L_lo=1, seed=2002),
+}
+
+
+def generate_mha(w: MhaWorkload, tail_fill: float = float("nan"), lengths: Optional[torch.Tensor] = None):
+    """Materialise (q [B,Sq,H,128], k [B,L,Hkv,128], v [B,L,Hkv,128], seqlens [B]) on the CPU."""
+    sl = w.lengths() if lengths is None else lengths.to(torch.int32)
+    q = torch.empty((w.B, w.Sq, w.H, MHA_D), dtype=torch.bfloat16)
+    k = torch.empty((w.B, w.L, w.Hkv, MHA_D), dtype=torch.bfloat16)
+    v = torch.empty((w.B, w.L, w.Hkv, MHA_D), dtype=torch.bfloat16)
+    for b in range(w.B):
+        gq = torch.Generator().manual_seed(_stream_seed(w.seed, b, 0))
+        q[b] = (torch.randn(w.Sq, w.H, MHA_D, generator=gq) * w.sigma).to(torch.bfloat16)
+        Lb = int(sl[b])
+        if Lb > 0:
+            gk = torch.Generator().manual_seed(_stream_seed(w.seed, b, 1))
+            gv = torch.Generator().manual_seed(_stream_seed(w.seed, b, 2))
+            k[b, :Lb] = (torch.randn(Lb, w.Hkv, MHA_D, generator=gk) * w.sigma).to(torch.bfloat16)
+            v[b, :Lb] = (torch.randn(Lb, w.Hkv, MHA_D, generator=gv) * w.sigma).to(torch.bfloat16)
+        if Lb < w.L:
+            k[b, Lb:] = tail_fill
+            v[b, Lb:] = tail_fill
+    return q, k, v, sl
+
+
 __all__ = ["Workload", "WORKLOADS", "generate", "make_q", "make_kv_rows", "small_variant",
-           "custom", "D_QK", "D_V", "D_ROPE", "ceil_div"]
+           "custom", "D_QK", "D_V", "D_ROPE", "ceil_div", "MhaWorkload", "MHA_WORKLOADS", "generate_mha", "MHA_D"]
