@@ -320,7 +320,8 @@ def run_ours(args, w: W.Workload):
         peak = peaks["bf16_tflops"]
         unit = "TFLOP/s"
     roof_time_ms = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e3
-    traffic, traffic_note = load_traffic(w.name)
+    # the record was taken with the default plan; a batch-invariant plan moves other bytes
+    traffic, traffic_note = load_traffic(w.name) if not plan.split_tiles else (None, None)
 
     cpu_base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -450,6 +451,7 @@ def run_mha(args, w: W.MhaWorkload):
         cpu_base = {"value": f_cpu / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
                     "sample": f"{nb} of {w.B} sequences, all query rows, {dt:.1f} s of fp64 CPU work"}
     achieved = nbytes / (main_ms * 1e-3) / 1e9
+    traffic, traffic_note = load_traffic(w.name)
     line = {
         "metric": f"MHA decode TFLOP/s + HBM GB/s at B={w.B},H={w.H},Hkv={w.Hkv},d=128,L={w.L}; fraction of roofline",
         "value": flops / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
@@ -462,7 +464,8 @@ def run_mha(args, w: W.MhaWorkload):
                    "l2": "inputs larger than L2, no flush"},
         "hbm_gbs": nbytes / (t_ms * 1e-3) / 1e9,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+                     "traffic_note": traffic_note,
                      "kernel": "mla_decode_transposed_kernel<G, MhaShape>", "kernel_ms": main_ms,
                      "combine_ms": comb_ms, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
                      "step_roofline_frac": nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3 / t_ms},
