@@ -12,6 +12,8 @@ cache, keys = 576-wide rows, values = their first 512 columns, natural-log LSE)
 is the one the TileLang pages use as their running example ("TileLang: Bridging
 Programmability and Performance in Modern Neural Kernels", papernotes.org,
 section "一个完整示例：FlashMLA 的两阶段优化"); the C file's header states it.
+``mla_decode_fp8`` is the same definition over a cache of E4M3 codes with one
+dequantization scale (the C file's FP8 section states the reading).
 """
 from __future__ import annotations
 
@@ -65,6 +67,11 @@ def _load():
             lib.oracle_mha_decode.restype = ctypes.c_int
             lib.oracle_mha_decode.argtypes = [ptr, ptr, ptr, ptr, i64, i64, i64, i64, i64, i64, i64,
                                               dbl, ptr, ptr, ctypes.c_int]
+            lib.oracle_mla_decode_fp8_rows.restype = ctypes.c_int
+            lib.oracle_mla_decode_fp8_rows.argtypes = [ptr, ptr, dbl, ptr, i64, i64, i64, i64, i64, i64,
+                                                       dbl, ptr, ptr, i64, ptr, ptr, ctypes.c_int]
+            lib.oracle_e4m3_to_double.restype = dbl
+            lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
             lib.oracle_max_threads.restype = ctypes.c_int
             lib.oracle_max_threads.argtypes = []
             _lib = lib
@@ -166,4 +173,61 @@ def mha_decode(q, k, v, seqlens, scale: float, num_threads: int = 0):
                                    out.ctypes.data, lse.ctypes.data, int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle_mha_decode failed with code {rc}")
+    return out, lse
+
+
+def _as_u8_codes(x) -> np.ndarray:
+    """E4M3 codes: a uint8 numpy array, or a torch uint8 / float8_e4m3fn tensor."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint8:
+            raise TypeError("numpy FP8 caches must hold E4M3 codes as uint8")
+        return np.ascontiguousarray(x)
+    import torch
+    if x.dtype == torch.float8_e4m3fn:
+        x = x.view(torch.uint8)
+    if x.dtype != torch.uint8:
+        raise TypeError(f"expected uint8 E4M3 codes, got {x.dtype}")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().numpy())
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Exact value of every E4M3 code (uint8 array-like), as float64."""
+    c = np.asarray(codes, dtype=np.uint8)
+    f = _load().oracle_e4m3_to_double
+    return np.array([f(int(v)) for v in c.reshape(-1)], dtype=np.float64).reshape(c.shape)
+
+
+def mla_decode_fp8(q, kv_codes, kv_scale: float, seqlens, scale: float, d_v: int = 512, num_threads: int = 0,
+                   sinks=None, row_ids=None):
+    """Oracle over an FP8 latent cache: kv value = kv_scale * e4m3(code).
+    q [B,Sq,H,d_qk] bf16, kv_codes [B,L_max,d_qk] uint8 (or float8_e4m3fn),
+    seqlens int [B], sinks None or [H].  row_ids None: every row, shapes
+    ([B,Sq,H,d_v], [B,Sq,H]); else the listed flattened rows r = (b*Sq + t)*H + h,
+    shapes ([n, d_v], [n])."""
+    qb = _as_bf16_bits(q)
+    kvc = _as_u8_codes(kv_codes)
+    if qb.ndim != 4 or kvc.ndim != 3:
+        raise ValueError("q must be [B,Sq,H,d_qk] and kv_codes [B,L_max,d_qk]")
+    B, Sq, H, d_qk = qb.shape
+    if kvc.shape[0] != B or kvc.shape[2] != d_qk:
+        raise ValueError("q and kv_codes disagree on B or d_qk")
+    L_max = kvc.shape[1]
+    sl = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
+    if sl.shape[0] != B:
+        raise ValueError("seqlens must have B entries")
+    if row_ids is None:
+        rows, rp, n = None, None, B * Sq * H
+        out = np.empty((B, Sq, H, d_v), dtype=np.float64)
+        lse = np.empty((B, Sq, H), dtype=np.float64)
+    else:
+        rows = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64).reshape(-1))
+        rp, n = rows.ctypes.data, rows.shape[0]
+        out = np.empty((n, d_v), dtype=np.float64)
+        lse = np.empty((n,), dtype=np.float64)
+    keep, sp = _sinks_arg(sinks, H)
+    rc = _load().oracle_mla_decode_fp8_rows(qb.ctypes.data, kvc.ctypes.data, float(kv_scale), sl.ctypes.data,
+                                            B, Sq, H, L_max, d_qk, d_v, float(scale), sp, rp, n,
+                                            out.ctypes.data, lse.ctypes.data, int(num_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_mla_decode_fp8_rows failed with code {rc}")
     return out, lse

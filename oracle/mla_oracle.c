@@ -47,7 +47,11 @@
  * identical keys, q = 0, two keys), invariants (permutation of keys, a shared
  * additive score shift, head and token independence), brute force in 50-digit
  * decimal arithmetic on tiny shapes, and torch's fp64 scaled_dot_product_
- * attention as an independent library routine.
+ * attention as an independent library routine.  The FP8-cache section at the
+ * end is pinned by the format's closed-form code values, torch's own E4M3
+ * decoding of all 256 codes, torch's fp64 attention over the dequantised
+ * cache, a single-key closed form, a scale-trade invariant, and equality with
+ * the bf16 definition when every value is exact in bf16.
  */
 #include <math.h>
 #include <stdint.h>
@@ -313,6 +317,131 @@ int oracle_mha_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
                 const int64_t h = r % H;
                 mha_one_row(q + r * D, k + b * L_max * Hkv * D, v + b * L_max * Hkv * Dv, seqlens[b], Hkv,
                             h / group, D, Dv, scale, scores, out + r * Dv, lse + r);
+            }
+            free(scores);
+        }
+    }
+    return failed ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * FP8 latent cache.  The same MLA decode, with the cache stored as 8-bit
+ * floating-point codes and one dequantization scale for the whole cache.
+ * The hackmd essay "TileLang 完整解析" (section "冷靜看待：TileLang 的局限與挑戰")
+ * names FP8 as the precision where TileLang's kernels trail or fail, and
+ * prints no format; the plain reading taken here is the common one for a
+ * quantized KV cache:
+ *
+ *   every element of kv[b, j, d] is an OCP "E4M3" code (1 sign bit, 4
+ *   exponent bits with bias 7, 3 mantissa bits; exponent field 0 encodes
+ *   subnormals (m / 8) 2^-6; S.1111.111 is NaN; there are no infinities;
+ *   largest finite magnitude 448), and the cached value is
+ *       kv_value = kv_scale * e4m3(code)
+ *   with kv_scale > 0 one fp32 number for the whole cache.
+ *
+ * The attention is then the definition at the top of this file applied to
+ * those values (sinks included): q stays bf16, keys are all 576 dequantized
+ * columns, values their first 512.  Arithmetic: each code is decoded exactly
+ * to double, multiplied by kv_scale in double (exact: 4 x 24 significand
+ * bits), and the rest is the same two-pass fp64 computation.
+ * ------------------------------------------------------------------------ */
+static double e4m3_to_double(uint8_t code)
+{
+    const int sign = code >> 7;
+    const int ex = (code >> 3) & 15;
+    const int man = code & 7;
+    double v;
+    if (ex == 15 && man == 7) return NAN;
+    if (ex == 0)
+        v = ldexp((double)man / 8.0, -6);           /* subnormal: 0.mmm x 2^(1 - 7) */
+    else
+        v = ldexp(1.0 + (double)man / 8.0, ex - 7); /* normal: 1.mmm x 2^(e - 7) */
+    return sign ? -v : v;
+}
+
+double oracle_e4m3_to_double(uint8_t code) { return e4m3_to_double(code); }
+
+/* One output row over an FP8 cache; as attend_one_row, with k_j[d] =
+ * kv_scale * e4m3(kv_seq[j, d]). */
+static void attend_one_row_fp8(const uint16_t *q_row, const uint8_t *kv_seq, double kv_scale,
+                               int64_t L, int64_t d_qk, int64_t d_v, double scale, double sink,
+                               double *scores, double *out_row, double *lse_out)
+{
+    if (L <= 0) {
+        for (int64_t e = 0; e < d_v; ++e) out_row[e] = 0.0;
+        *lse_out = sink;
+        return;
+    }
+    for (int64_t j = 0; j < L; ++j) {
+        const uint8_t *k_row = kv_seq + j * d_qk;
+        double dot = 0.0;
+        for (int64_t d = 0; d < d_qk; ++d)
+            dot += bf16_bits_to_double(q_row[d]) * (kv_scale * e4m3_to_double(k_row[d]));
+        scores[j] = scale * dot;
+    }
+    double m = scores[0];
+    for (int64_t j = 1; j < L; ++j)
+        if (scores[j] > m) m = scores[j];
+    if (sink > m) m = sink;
+    double l = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+        scores[j] = exp(scores[j] - m);
+        l += scores[j];
+    }
+    l += exp(sink - m);
+    for (int64_t e = 0; e < d_v; ++e) out_row[e] = 0.0;
+    for (int64_t j = 0; j < L; ++j) {
+        const uint8_t *v_row = kv_seq + j * d_qk;
+        const double w = scores[j];
+        for (int64_t e = 0; e < d_v; ++e)
+            out_row[e] += w * (kv_scale * e4m3_to_double(v_row[e]));
+    }
+    for (int64_t e = 0; e < d_v; ++e) out_row[e] /= l;
+    *lse_out = m + log(l);
+}
+
+/*
+ * FP8-cache oracle for caller-chosen flattened rows r = (b * Sq + t) * H + h
+ * (row_ids = NULL: every row, in order, n_rows ignored).
+ *   q : bf16 bits [B, Sq, H, d_qk];  kv : E4M3 codes [B, L_max, d_qk]
+ *   kv_scale : the cache's dequantization scale;  sinks : double [H] or NULL
+ *   out : double [n, d_v];  lse : double [n]
+ */
+int oracle_mla_decode_fp8_rows(const uint16_t *q, const uint8_t *kv, double kv_scale, const int32_t *seqlens,
+                               int64_t B, int64_t Sq, int64_t H, int64_t L_max,
+                               int64_t d_qk, int64_t d_v, double scale, const double *sinks,
+                               const int64_t *row_ids, int64_t n_rows,
+                               double *out, double *lse, int num_threads)
+{
+    if (!q || !kv || !seqlens || !out || !lse) return -1;
+    if (B < 0 || Sq < 1 || H < 1 || L_max < 0 || d_qk < 1 || d_v < 1 || d_v > d_qk) return -1;
+    if (!isfinite(kv_scale)) return -1;
+    const int64_t all = B * Sq * H;
+    if (!row_ids) n_rows = all;
+    for (int64_t i = 0; row_ids && i < n_rows; ++i)
+        if (row_ids[i] < 0 || row_ids[i] >= all) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > L_max) return -1;
+    int failed = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+#pragma omp parallel
+    {
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(L_max > 0 ? L_max : 1));
+        if (!scores) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int64_t i = 0; i < n_rows; ++i) {
+                const int64_t r = row_ids ? row_ids[i] : i;
+                const int64_t b = r / (Sq * H);
+                const double sink = sinks ? sinks[r % H] : -INFINITY;
+                attend_one_row_fp8(q + r * d_qk, kv + b * L_max * d_qk, kv_scale, seqlens[b],
+                                   d_qk, d_v, scale, sink, scores, out + i * d_v, lse + i);
             }
             free(scores);
         }

@@ -382,3 +382,127 @@ def pin_mha_single_key(impl):
 
 
 MHA_PINS = [pin_mha_mqa_equals_latent_definition, pin_mha_sdpa_library, pin_mha_head_groups, pin_mha_single_key]
+
+
+# ---------------------------------------------------------------- FP8 latent cache
+# FP8 pins take (decode, attend): decode(codes uint8 array) -> float64 values
+# of the E4M3 codes; attend(q, codes, kv_scale, seqlens, scale, d_v, sinks)
+# -> (out, lse) for a cache of codes whose values are kv_scale * e4m3(code).
+
+def _codes_from_normal(shape, gen, sigma, kv_scale):
+    """Random E4M3 codes of N(0, sigma) values quantised with kv_scale (torch's
+    own rounding; this only makes inputs)."""
+    x = torch.randn(*shape, generator=gen, dtype=torch.float64) * sigma / kv_scale
+    return x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _torch_e4m3_values(codes):
+    return codes.view(torch.float8_e4m3fn).to(torch.float64)
+
+
+def pin_fp8_decode_library(decode, attend):
+    """All 256 codes against torch's float8_e4m3fn -> float64 conversion (an
+    independent library routine); the two NaN codes must decode to NaN."""
+    codes = np.arange(256, dtype=np.uint8)
+    got = decode(codes)
+    ref = _torch_e4m3_values(torch.from_numpy(codes)).numpy()
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    fin = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[fin], ref[fin])
+    np.testing.assert_array_equal(np.signbit(got[fin]), np.signbit(ref[fin]))
+
+
+def pin_fp8_decode_closed_forms(decode, attend):
+    """Values fixed by the format: 1 sign, 4 exponent bits (bias 7), 3 mantissa
+    bits, subnormals (m/8) 2^-6 at exponent field 0, S.1111.111 = NaN."""
+    table = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x0F: 1.875 * 2.0 ** -6,
+             0x38: 1.0, 0x3F: 1.875, 0x40: 2.0, 0x77: 240.0, 0x7E: 448.0, 0x80: -0.0, 0xB8: -1.0,
+             0xFE: -448.0, 0x81: -(2.0 ** -9)}
+    got = decode(np.array(sorted(table), dtype=np.uint8))
+    for v, (c, want) in zip(got, sorted(table.items())):
+        assert v == want and math.copysign(1.0, v) == math.copysign(1.0, want), (hex(c), v, want)
+    assert np.isnan(decode(np.array([0x7F, 0xFF], dtype=np.uint8))).all()
+
+
+def pin_fp8_sdpa_library(decode, attend):
+    """torch's fp64 scaled_dot_product_attention over the dequantised cache
+    (kv_scale * torch's own E4M3 values; keys all 576 columns, values the
+    first 512) and torch.logsumexp, with a scale that is not a power of two,
+    ragged lengths and two tokens."""
+    g = torch.Generator().manual_seed(61)
+    ks = 0.0123
+    q = _rand_bf16((2, 2, 4, 576), g)
+    codes = _codes_from_normal((2, 53, 576), g, 1.0, ks)
+    sl = np.array([53, 19], np.int32)
+    out, lse = attend(q, codes, ks, sl, SCALE, 512, None)
+    kvd = _torch_e4m3_values(codes) * ks
+    for b in range(2):
+        L = int(sl[b])
+        qq = q[b].double().reshape(1, -1, 576)
+        kk = kvd[b, :L].reshape(1, L, 576)
+        vv = kvd[b, :L, :512].reshape(1, L, 512)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, scale=SCALE)
+        np.testing.assert_allclose(out[b].reshape(-1, 512), ref[0].numpy(), rtol=0, atol=1e-12)
+        sc = (qq[0] @ kk[0].T) * SCALE
+        np.testing.assert_allclose(lse[b].reshape(-1), torch.logsumexp(sc, dim=-1).numpy(), rtol=0, atol=1e-12)
+
+
+def pin_fp8_single_key(decode, attend):
+    """L = 1: out is the key's dequantised value row (kv_scale * e4m3), exactly;
+    lse is its scaled score."""
+    g = torch.Generator().manual_seed(62)
+    ks = 0.037
+    q = _rand_bf16((1, 1, 3, 576), g)
+    codes = _codes_from_normal((1, 2, 576), g, 1.0, ks)
+    out, lse = attend(q, codes, ks, np.array([1], np.int32), SCALE, 512, None)
+    vals = _torch_e4m3_values(codes[0, 0]) * ks
+    for h in range(3):
+        np.testing.assert_array_equal(out[0, 0, h], vals[:512].numpy())
+        s0 = SCALE * float(torch.dot(q[0, 0, h].double(), vals))
+        assert abs(lse[0, 0, h] - s0) <= 1e-12 * max(1.0, abs(s0))
+
+
+def pin_fp8_scale_trade(decode, attend):
+    """Doubling kv_scale while halving the softmax scale leaves every score,
+    hence the weights and lse, unchanged and doubles every value: out doubles."""
+    g = torch.Generator().manual_seed(63)
+    ks = 0.02
+    q = _rand_bf16((2, 1, 3, 576), g)
+    codes = _codes_from_normal((2, 31, 576), g, 1.0, ks)
+    sl = np.array([31, 8], np.int32)
+    o1, l1 = attend(q, codes, ks, sl, 0.08, 512, None)
+    o2, l2 = attend(q, codes, 2 * ks, sl, 0.04, 512, None)
+    np.testing.assert_allclose(o2, 2 * o1, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(l2, l1, rtol=1e-13, atol=1e-13)
+
+
+def pin_fp8_all_codes_equal_bf16_cache(decode, attend):
+    """Every finite code, with a power-of-two kv_scale (2^-7), gives values that
+    bf16 holds exactly, so the FP8 definition must reproduce the (separately
+    pinned) bf16-cache oracle on that bf16 cache -- sinks, an empty sequence
+    and a ragged length included -- up to summation order (the oracle itself
+    matches bit for bit: tests/test_oracle.py)."""
+    import oracle  # the bf16 definition, pinned by ALL_PINS and SINK_PINS
+    g = torch.Generator().manual_seed(64)
+    finite = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    B, L = 3, 40
+    codes = np.empty((B, L, 576), dtype=np.uint8)
+    rng = np.random.default_rng(64)
+    for b in range(B):
+        for j in range(L):
+            codes[b, j] = rng.choice(finite, size=576)
+    ks = 2.0 ** -7
+    q = _rand_bf16((B, 2, 2, 576), g, sigma=0.05)
+    sl = np.array([40, 0, 23], np.int32)
+    sinks = np.array([0.3, -2.0])
+    codes_t = torch.from_numpy(codes)
+    kv_bf16 = (_torch_e4m3_values(codes_t) * ks).to(torch.bfloat16)
+    assert torch.equal(kv_bf16.double(), _torch_e4m3_values(codes_t) * ks)  # exact in bf16
+    out, lse = attend(q, codes_t, ks, sl, SCALE, 512, sinks)
+    ro, rl = oracle.mla_decode(q, kv_bf16, sl, SCALE, sinks=sinks)
+    np.testing.assert_allclose(out, ro, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, rl, rtol=0, atol=1e-13)
+
+
+FP8_PINS = [pin_fp8_decode_library, pin_fp8_decode_closed_forms, pin_fp8_sdpa_library, pin_fp8_single_key,
+            pin_fp8_scale_trade, pin_fp8_all_codes_equal_bf16_cache]

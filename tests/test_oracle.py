@@ -253,3 +253,129 @@ def test_mha_pins_catch_planted_mistakes(name):
         assert failed == [], f"a correct stand-in must pass every MHA pin, failed: {failed}"
     else:
         assert failed, f"planted mistake '{name}' passed every MHA pin"
+
+
+# ---------------------------------------------------------------- FP8 latent cache oracle
+
+def _oracle_fp8_attend(q, codes, ks, sl, scale, d_v, sinks):
+    return oracle.mla_decode_fp8(q, codes, ks, sl, scale, d_v=d_v, sinks=sinks)
+
+
+@pytest.mark.parametrize("pin", pins.FP8_PINS, ids=lambda p: p.__name__)
+def test_fp8_oracle_pin(pin):
+    pin(oracle.e4m3_decode, _oracle_fp8_attend)
+
+
+def test_fp8_rows_entry_matches_full():
+    g = torch.Generator().manual_seed(65)
+    q = torch.randn(2, 2, 3, 576, generator=g).to(torch.bfloat16)
+    codes = (torch.randn(2, 21, 576, generator=g) * 20).to(torch.float8_e4m3fn).view(torch.uint8)
+    sl = np.array([21, 0], np.int32)
+    sinks = np.array([0.5, -1.0, 3.0])
+    out, lse = oracle.mla_decode_fp8(q, codes, 0.05, sl, pins.SCALE, sinks=sinks)
+    rows = np.array([0, 4, 7, 11, 5])
+    o2, l2 = oracle.mla_decode_fp8(q, codes, 0.05, sl, pins.SCALE, sinks=sinks, row_ids=rows)
+    np.testing.assert_array_equal(o2, out.reshape(-1, 512)[rows])
+    np.testing.assert_array_equal(l2, lse.reshape(-1)[rows])
+
+
+def test_fp8_oracle_is_the_bf16_oracle_on_exact_values():
+    """Same operations in the same order on the same doubles: bit-identical."""
+    g = torch.Generator().manual_seed(66)
+    codes = torch.randint(0, 256, (2, 33, 576), generator=g, dtype=torch.uint8)
+    codes[(codes == 0x7F) | (codes == 0xFF)] = 0x7E
+    q = (torch.randn(2, 1, 4, 576, generator=g) * 0.05).to(torch.bfloat16)
+    sl = np.array([33, 9], np.int32)
+    ks = 2.0 ** -6
+    kv = (codes.view(torch.float8_e4m3fn).to(torch.float64) * ks).to(torch.bfloat16)
+    out, lse = oracle.mla_decode_fp8(q, codes, ks, sl, pins.SCALE)
+    ro, rl = oracle.mla_decode(q, kv, sl, pins.SCALE)
+    np.testing.assert_array_equal(out, ro)
+    np.testing.assert_array_equal(lse, rl)
+
+
+def test_fp8_rejects_non_finite_scale():
+    q = torch.zeros(1, 1, 1, 576, dtype=torch.bfloat16)
+    codes = np.zeros((1, 4, 576), np.uint8)
+    with pytest.raises(ValueError):
+        oracle.mla_decode_fp8(q, codes, float("nan"), np.array([4], np.int32), 0.1)
+
+
+def _np_e4m3(codes, *, bias=7, subnormal_as_normal=False, sign=True, man_bits=3, nan_code=True):
+    c = np.asarray(codes, dtype=np.int64)
+    s = c >> 7
+    e = (c >> 3) & 15
+    m = (c & 7).astype(np.float64)
+    frac = m / (2 ** man_bits)
+    if subnormal_as_normal:
+        v = (1.0 + frac) * np.exp2(np.maximum(e, 1) - bias)
+    else:
+        v = np.where(e == 0, frac * 2.0 ** (1 - bias), (1.0 + frac) * np.exp2(e - bias))
+    if sign:
+        v = np.where(s == 1, -v, v)
+    if nan_code:
+        v = np.where((e == 15) & (c & 7 == 7), np.nan, v)
+    return v
+
+
+def _np_fp8_attend(q, codes, ks, sl, scale, d_v, sinks, *, dec=None, ks_keys="mul", ks_values="mul"):
+    dec = dec or {}
+    vals = _np_e4m3(np.asarray(codes), **dec)
+    kscale = {"mul": ks, "none": 1.0, "div": 1.0 / ks}
+    kd = vals * kscale[ks_keys]
+    vd = vals[..., :d_v] * kscale[ks_values]
+    qd = q.to(torch.float64).numpy()
+    B, Sq, H, _ = qd.shape
+    out = np.zeros((B, Sq, H, d_v))
+    lse = np.zeros((B, Sq, H))
+    for b in range(B):
+        L = int(sl[b])
+        for t in range(Sq):
+            for h in range(H):
+                sg = -np.inf if sinks is None else float(sinks[h])
+                if L == 0:
+                    lse[b, t, h] = sg
+                    continue
+                s = (kd[b, :L] @ qd[b, t, h]) * scale
+                m = max(s.max(), sg)
+                w = np.exp(s - m)
+                l = w.sum() + np.exp(sg - m)
+                out[b, t, h] = (w @ vd[b, :L]) / l
+                lse[b, t, h] = m + np.log(l)
+    return out, lse
+
+
+FP8_MUTANTS = {
+    "correct": {},
+    "exponent_bias_8": dict(dec=dict(bias=8)),
+    "subnormals_read_as_normals": dict(dec=dict(subnormal_as_normal=True)),
+    "sign_bit_ignored": dict(dec=dict(sign=False)),
+    "mantissa_read_as_4_bits": dict(dec=dict(man_bits=4)),
+    "nan_code_read_as_finite": dict(dec=dict(nan_code=False)),
+    "kv_scale_not_on_keys": dict(ks_keys="none"),
+    "kv_scale_not_on_values": dict(ks_values="none"),
+    "kv_scale_divides": dict(ks_keys="div", ks_values="div"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FP8_MUTANTS))
+def test_fp8_pins_catch_planted_mistakes(name):
+    kw = FP8_MUTANTS[name]
+
+    def decode(codes):
+        return _np_e4m3(codes, **kw.get("dec", {}))
+
+    def attend(q, codes, ks, sl, scale, d_v, sinks):
+        return _np_fp8_attend(q, codes, ks, sl, scale, d_v, sinks, **kw)
+
+    failed = []
+    for pin in pins.FP8_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(decode, attend)
+        except AssertionError:
+            failed.append(pin.__name__)
+    if name == "correct":
+        assert failed == [], f"a correct stand-in must pass every FP8 pin, failed: {failed}"
+    else:
+        assert failed, f"planted mistake '{name}' passed every FP8 pin"
