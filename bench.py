@@ -479,6 +479,128 @@ def run_mha(args, w: W.MhaWorkload):
     print(json.dumps(line), flush=True)
 
 
+def run_fp8(args, w: W.Workload):
+    """MLA decode over an FP8 (E4M3) latent cache: same timing rules as
+    run_ours (graph replay, per-kernel graphs, host-buffer e2e), one GPU."""
+    from mla_decode_attention_11_b200 import binding as M
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    q, codes, ks, sl = W.generate_fp8(w)
+    qd, cd, sld = q.to(dev), codes.to(dev), sl.to(dev)
+    plan = M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=0)
+    ws = M.alloc_workspace(plan, device=dev)
+    M.mla_decode_workspace_init(plan, ws)
+    out = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Sq, w.H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(dev)
+
+    def step():
+        M.mla_decode_run_fp8(plan, qd, cd, ks, sld, w.scale, out, lse, ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    M.mla_decode_check(plan, ws, stream=stream)
+
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(n):
+                    fn()
+        return g
+
+    def replay_ms(g, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / n
+
+    g_steps = capture(step, args.steps)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(0)
+    clocks.start()
+    t_ms = replay_ms(g_steps, args.steps)
+    clk = clocks.stop()
+    del g_steps
+    n_brk = max(3, min(args.steps, 50))
+    main_ms = replay_ms(capture(lambda: M.mla_decode_run_fp8_phase(plan, qd, cd, ks, sld, w.scale, out, lse, ws, 1,
+                                                                   stream=stream), n_brk), n_brk)
+    comb_ms = replay_ms(capture(lambda: M.mla_decode_run_fp8_phase(plan, qd, cd, ks, sld, w.scale, out, lse, ws, 2,
+                                                                   stream=stream), n_brk), n_brk)
+    M.mla_decode_check(plan, ws, stream=stream)
+    # end to end: host buffers in, host buffers out, copies inside the timed region
+    qh, ch, slh = q.pin_memory(), codes.pin_memory(), sl.pin_memory()
+    outh = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 5))
+    with torch.cuda.stream(stream):
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            qd.copy_(qh, non_blocking=True)
+            cd.copy_(ch, non_blocking=True)
+            sld.copy_(slh, non_blocking=True)
+            step()
+            outh.copy_(out, non_blocking=True)
+            lseh.copy_(lse, non_blocking=True)
+        f1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = f0.elapsed_time(f1) / e2e_steps
+    M.mla_decode_check(plan, ws, stream=stream)
+    flops, nbytes = w.algorithmic_flops(sl), w.algorithmic_bytes_fp8(sl)
+    peaks, peak_src = load_peaks()
+    cpu_base = None
+    if not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        R = w.Sq * w.H
+        b0 = 0
+        rows = np.arange(b0 * R, (b0 + 1) * R, dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.mla_decode_fp8(q, codes, ks, sl, w.scale, row_ids=rows)
+        dt = time.perf_counter() - t0
+        f_cpu = int(sl[b0]) * R * 2 * (W.D_QK + W.D_V)
+        cpu_base = {"value": f_cpu / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
+                    "sample": f"1 of {w.B} sequences, all {R} query rows, {dt:.1f} s of fp64 CPU work"}
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    bound = "hbm" if flops / nbytes < ridge else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = nbytes / (main_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:  # f16 MMAs: the measured bf16 figure (same dense rate)
+        achieved, peak, unit = flops / (main_ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    traffic, traffic_note = load_traffic(w.name + "_fp8")
+    line = {
+        "metric": METRIC + " (FP8 latent cache)",
+        "value": flops / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 cache, f16 MMA", "data": "synthetic",
+        "config": {"workload": workload_desc(w) + f"; cache quantised to E4M3, kv_scale = amax/448 = {ks:.6g}",
+                   "global_batch": w.B, "seq_len": w.L, "parallelism": "single GPU", "kernel": "transposed (FP8)",
+                   "group_rows": plan.group_rows, "partitions": plan.num_partitions,
+                   "l2": "inputs larger than L2 (kv %.0f MB > 126 MB), no flush" % (codes.numel() / 1e6)},
+        "hbm_gbs": nbytes / (t_ms * 1e-3) / 1e9,
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                     "traffic_note": traffic_note,
+                     "kernel": "mla_decode_transposed_kernel<G, MlaFp8Shape>", "kernel_ms": main_ms,
+                     "combine_ms": comb_ms, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                     "hbm_frac": nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "step_roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
+                                               flops / (peaks["bf16_tflops"] * 1e12)) * 1e3 / t_ms},
+        "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": q.numel() * 2 + codes.numel() + sl.numel() * 4,
+                "d2h_bytes_per_step": out.numel() * 2 + lse.numel() * 4, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+        "cpu_baseline": cpu_base,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -491,6 +613,8 @@ def main():
                     help="use the batch-invariant plan, sequences cut every SPLIT_TILES KV tiles (0 = default)")
     ap.add_argument("--sinks", action="store_true",
                     help="time the attention-sink entry point (per-head sink logits) on the same workload")
+    ap.add_argument("--fp8", action="store_true",
+                    help="the same MLA workload over an FP8 (E4M3) latent cache (mla_decode_run_fp8)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -501,6 +625,12 @@ def main():
         run_mha(args, W.MHA_WORKLOADS[args.workload])
         return
     w = W.WORKLOADS[args.workload]
+    if args.fp8:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm covers the bf16 cache"}))
+            return
+        run_fp8(args, w)
+        return
     if args.impl == "reference":
         run_reference(args, w)
     else:

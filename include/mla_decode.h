@@ -62,7 +62,9 @@ typedef enum mla_status {
 enum {
     MLA_KERNEL_TRANSPOSED = 1, /* S^T = K Q^T per CTA, kv rows on the 128 TMEM lanes (any H*Sq) */
     MLA_KERNEL_PAIR = 2,       /* CTA pair, 64 query rows per CTA, cta_group::2 MMAs (H*Sq % 128 == 0) */
-    MLA_KERNEL_MHA = 3         /* MHA decode (mha_decode_plan): the transposed kernel over 128-wide K, V */
+    MLA_KERNEL_MHA = 3,        /* MHA decode (mha_decode_plan): the transposed kernel over 128-wide K, V */
+    MLA_KERNEL_FP8 = 4         /* MLA decode over an FP8 cache (mla_decode_plan_fp8): the transposed kernel
+                                  with E4M3 chunks widened to f16 in shared memory */
 };
 
 /*
@@ -322,6 +324,57 @@ mla_status mha_decode_run(const mla_plan* plan, const void* q, const void* k, co
 mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void* k, const void* v,
                                 const int32_t* seqlens, float softmax_scale, const float* sinks, void* out, float* lse,
                                 void* workspace, size_t workspace_bytes, void* stream, int32_t phase);
+
+/*
+ * FP8 latent cache.  The hackmd essay "TileLang 完整解析" (section "冷靜看待：
+ * TileLang 的局限與挑戰") names FP8 as the precision where TileLang trails or
+ * fails and prints no format; this library takes the common reading of an
+ * FP8 KV cache: every element of the [B, L_max, 576] cache is an OCP E4M3
+ * code (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, subnormals
+ * at exponent 0, S.1111.111 = NaN, largest finite 448) and
+ *     kv_value[b, j, d] = kv_scale * e4m3(kv_fp8[b, j, d])
+ * with one fp32 kv_scale for the whole cache.  The decode is the definition
+ * at the top of this file on those values (keys: all 576 columns; values:
+ * the first 512), with q bf16, out bf16 and lse fp32 as there.
+ *
+ * Numerics: every E4M3 value divided by 2^8 is exact in f16, so the kernel
+ * widens the codes to those f16 values in shared memory (integer bit moves)
+ * and runs f16 x f16 -> f32 tensor-core MMAs; q is narrowed from bf16 to f16
+ * (exact for 2^-17 <= |q| <= 65504; |q| > 65504 becomes inf, smaller |q| lose
+ * at most 2^-25), P is rounded to f16, and kv_scale * 2^8 multiplies the
+ * scores (with softmax_scale) and the output rows.
+ *
+ * mla_decode_plan_fp8 -- as mla_decode_plan (same arguments, limits and return
+ * codes) for an FP8 cache; the plan's kernel is MLA_KERNEL_FP8 (the transposed
+ * kernel, 16 or 32 query rows per CTA, 320 threads), for every head count.
+ */
+mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                               int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
+
+/*
+ * mla_decode_run_fp8 -- enqueue one MLA decode over an FP8 cache on `stream`.
+ *   plan     from mla_decode_plan_fp8 (any other plan: MLA_ERR_INVALID_ARG)
+ *   q        device, bf16 [B, Sq, H, 576], contiguous, 16-byte aligned
+ *   kv_fp8   device, E4M3 codes (one byte each) [B, L_max, 576], contiguous,
+ *            16-byte aligned; rows at or past seqlens[b] are never used
+ *   kv_scale the cache's dequantization scale, finite and > 0
+ *            (else MLA_ERR_INVALID_ARG)
+ *   seqlens, softmax_scale, out, lse, workspace, workspace_bytes, stream
+ *            as mla_decode_run;  sinks as mla_decode_run_sinks (NULL = none)
+ * Launches the main kernel and the split-KV combine; no host sync, no
+ * allocation; return codes as mla_decode_run.  The cache must hold finite
+ * codes: the two NaN codes (S.1111.111) are read as +-480 (times kv_scale),
+ * not as NaN.
+ */
+mla_status mla_decode_run_fp8(const mla_plan* plan, const void* q, const void* kv_fp8, float kv_scale,
+                              const int32_t* seqlens, float softmax_scale, const float* sinks, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* mla_decode_run_fp8_phase -- the launches of mla_decode_run_fp8 (no sinks) one
+ * at a time (1 = main kernel, 2 = split-KV combine), as mla_decode_run_phase. */
+mla_status mla_decode_run_fp8_phase(const mla_plan* plan, const void* q, const void* kv_fp8, float kv_scale,
+                                    const int32_t* seqlens, float softmax_scale, void* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, void* stream, int32_t phase);
 
 /* Static English description of a status code (never NULL). */
 const char* mla_status_string(mla_status status);

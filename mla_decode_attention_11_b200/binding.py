@@ -33,13 +33,15 @@ STATUS_NAMES = {0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_ALIGNMENT", 3
 MLA_KERNEL_TRANSPOSED = 1
 MLA_KERNEL_PAIR = 2
 MLA_KERNEL_MHA = 3
+MLA_KERNEL_FP8 = 4
 MHA_D = 128
 MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
 EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_plan_batch_invariant", "mla_decode_workspace_init", "mla_decode_run", "mla_decode_run_phase",
                     "mla_decode_check", "mla_decode_run_noalloc", "mla_decode_run_sinks",
                     "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug",
-                    "mha_decode_plan", "mha_decode_run", "mha_decode_run_phase")
+                    "mha_decode_plan", "mha_decode_run", "mha_decode_run_phase",
+                    "mla_decode_plan_fp8", "mla_decode_run_fp8", "mla_decode_run_fp8_phase")
 
 
 class MlaError(RuntimeError):
@@ -115,6 +117,15 @@ def load_library(build_if_missing: bool = True):
         lib.mha_decode_run_phase.restype = c_i32
         lib.mha_decode_run_phase.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_vp, c_vp, c_f, c_vp, c_vp, c_vp,
                                              c_vp, c_sz, c_vp, c_i32]
+        lib.mla_decode_plan_fp8.restype = c_i32
+        lib.mla_decode_plan_fp8.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(mla_plan),
+                                            ctypes.POINTER(c_sz)]
+        lib.mla_decode_run_fp8.restype = c_i32
+        lib.mla_decode_run_fp8.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_f, c_vp, c_f, c_vp, c_vp, c_vp,
+                                           c_vp, c_sz, c_vp]
+        lib.mla_decode_run_fp8_phase.restype = c_i32
+        lib.mla_decode_run_fp8_phase.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_f, c_vp, c_f, c_vp, c_vp,
+                                                 c_vp, c_sz, c_vp, c_i32]
         lib.mla_decode_check.restype = c_i32
         lib.mla_decode_check.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp]
         lib.mla_status_string.restype = ctypes.c_char_p
@@ -385,3 +396,61 @@ def mha_decode_run_phase(plan: mla_plan, q, k, v, seqlens, softmax_scale: float,
                                              _stream_handle(stream), int(phase))
     if rc != MLA_OK:
         raise MlaError(rc, "mha_decode_run_phase")
+
+
+# ---------------------------------------------------------------- FP8 latent cache
+
+def mla_decode_plan_fp8(B: int, Sq: int, H: int, L_max: int, device: Optional[int] = None,
+                        num_partitions: int = 0) -> mla_plan:
+    """A plan for a cache of E4M3 codes (mla_decode_plan_fp8): the transposed
+    kernel with FP8 staging, for every head count."""
+    if device is None:
+        device = torch.cuda.current_device()
+    p = mla_plan()
+    ws = ctypes.c_size_t(0)
+    rc = load_library().mla_decode_plan_fp8(int(B), int(Sq), int(H), int(L_max), int(device), int(num_partitions),
+                                            ctypes.byref(p), ctypes.byref(ws))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mla_decode_plan_fp8")
+    return p
+
+
+def _fp8_codes(kv_fp8: torch.Tensor) -> torch.Tensor:
+    return kv_fp8.view(torch.uint8) if kv_fp8.dtype == torch.float8_e4m3fn else kv_fp8
+
+
+def mla_decode_run_fp8(plan: mla_plan, q: torch.Tensor, kv_fp8: torch.Tensor, kv_scale: float,
+                       seqlens: torch.Tensor, softmax_scale: float, out: torch.Tensor, lse: torch.Tensor,
+                       workspace: torch.Tensor, sinks: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Enqueue one decode over an FP8 cache: kv_fp8 is a CUDA tensor of E4M3
+    codes [B, L_max, 576] (torch.uint8 or torch.float8_e4m3fn), kv_value =
+    kv_scale * e4m3(code); sinks as in mla_decode_run_sinks."""
+    B, Sq, H, L = plan.B, plan.Sq, plan.H, plan.L_max
+    codes = _fp8_codes(kv_fp8)
+    _check_tensor(q, "q", torch.bfloat16, (B, Sq, H, D_QK))
+    _check_tensor(codes, "kv_fp8", torch.uint8, (B, L, D_QK))
+    _check_tensor(seqlens, "seqlens", torch.int32, (B,))
+    _check_tensor(out, "out", torch.bfloat16, (B, Sq, H, D_V))
+    _check_tensor(lse, "lse", torch.float32, (B, Sq, H))
+    if sinks is not None:
+        _check_tensor(sinks, "sinks", torch.float32, (H,))
+    rc = load_library().mla_decode_run_fp8(ctypes.byref(plan), q.data_ptr(), codes.data_ptr(), float(kv_scale),
+                                           seqlens.data_ptr(), float(softmax_scale),
+                                           sinks.data_ptr() if sinks is not None else None, out.data_ptr(),
+                                           lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                           _stream_handle(stream))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mla_decode_run_fp8")
+
+
+def mla_decode_run_fp8_phase(plan: mla_plan, q: torch.Tensor, kv_fp8: torch.Tensor, kv_scale: float,
+                             seqlens: torch.Tensor, softmax_scale: float, out: torch.Tensor, lse: torch.Tensor,
+                             workspace: torch.Tensor, phase: int, stream=None) -> None:
+    """One of the two launches of mla_decode_run_fp8 (1 = main kernel, 2 = combine)."""
+    codes = _fp8_codes(kv_fp8)
+    rc = load_library().mla_decode_run_fp8_phase(ctypes.byref(plan), q.data_ptr(), codes.data_ptr(),
+                                                 float(kv_scale), seqlens.data_ptr(), float(softmax_scale),
+                                                 out.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                                 workspace.numel(), _stream_handle(stream), int(phase))
+    if rc != MLA_OK:
+        raise MlaError(rc, "mla_decode_run_fp8_phase")

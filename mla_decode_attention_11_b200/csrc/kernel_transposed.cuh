@@ -18,22 +18,27 @@
 // section "三大核心優化機制": a TMA producer warp and consumer warps joined by
 // mbarriers), with one warp issuing all tcgen05 MMAs.
 //
-// Warp roles (192 threads):
+// Warp roles (192 threads; 320 with an FP8 cache):
 //   warps 0-3  softmax + epilogue (thread = TMEM lane = kv row / dv row)
 //   warp 4     TMA producer (one elected lane)
 //   warp 5     TMEM allocator + MMA issuer (one elected lane)
+//   warps 6-9  FP8 cache only (6-7 at G = 32): widen staged E4M3 chunks to f16
+//              operands (thread = kv row), and Q from bf16 to f16 once per piece
 //
 // Shared memory (1024-byte aligned regions, 128-byte swizzle for TMA data):
 //   pair ring  NP x 32 KB: a [128 kv x 128 col] block = dv chunks 2p, 2p+1
 //   rope ring  NR x 16 KB: the [128 kv x 64] rope chunk (columns 512..575)
 //   Q          9 x [G x 64] chunks, loaded once per piece
-//   P^T        [128 kv x G] bf16, MN-major (q contiguous), 32/64-byte swizzle
+//   P^T        [128 kv x G] bf16 (f16 with an FP8 cache), MN-major (q contiguous),
+//              32/64-byte swizzle
+//   FP8 ring   NF x 8 KB: [128 kv x 64] E4M3 codes, 64-byte swizzle (FP8 cache only)
 // Every pipeline wait is bounded (%globaltimer); on expiry the CTA records
 // kStatusTimeout, drains its own TMA loads and MMAs, frees TMEM and returns.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -62,20 +67,36 @@ struct MainArgs {
     int split_tiles;     // 0: balanced schedule; > 0: batch-invariant chunks of this many tiles
     int Sq;              // query tokens per sequence
     int Hkv;             // MHA: kv heads (query head h reads kv head h / (H / Hkv)); MLA: 1
+    float o_scale;       // factor on every output row: the FP8 cache's kv_scale, else 1
 };
 
 // The two attention shapes the transposed kernel serves.
 struct MlaShape {  // latent cache: keys are 576-wide kv rows, values their first 512 columns
     static constexpr bool kMha = false;
+    static constexpr bool kFp8 = false;
     static constexpr int kQKChunks = 9;  // 64-column chunks of a key (chunk 8 = rope)
     static constexpr int kDvBlocks = 4;  // 128-wide blocks of a value row
     static constexpr int kDv = 512;
 };
 struct MhaShape {  // multi-head attention: separate K and V tensors, 128 wide, grouped kv heads
     static constexpr bool kMha = true;
+    static constexpr bool kFp8 = false;
     static constexpr int kQKChunks = 2;
     static constexpr int kDvBlocks = 1;
     static constexpr int kDv = 128;
+};
+// The latent cache stored as E4M3 codes with one dequantization scale: each
+// 64-column chunk is staged as 8 KB of codes, widened to f16 in shared memory
+// by the converter warps (every E4M3 value, divided by 2^8, is exact in f16),
+// and the MMAs run kind::f16 on f16 operands (Q is narrowed from bf16 to f16
+// once per piece, P^T is written as f16).  kv_scale * 2^8 enters the score
+// scale and o_scale.
+struct MlaFp8Shape {
+    static constexpr bool kMha = false;
+    static constexpr bool kFp8 = true;
+    static constexpr int kQKChunks = 9;
+    static constexpr int kDvBlocks = 4;
+    static constexpr int kDv = 512;
 };
 
 // Folds a per-head attention sink into a finished row.  (m, l) are the row's
@@ -94,28 +115,43 @@ __device__ __forceinline__ float fold_sink(float& m, float& l, float s2) {
 
 constexpr float kLog2e = 1.4426950408889634074f;
 
+// FP8 cache at G = 16: operand pair slots and 8-KB staging slots (5 + 3 fill
+// the shared memory; a pair slot can be traded for four staging slots)
+#ifndef MLA_FP8_NP16
+#define MLA_FP8_NP16 5
+#endif
+#ifndef MLA_FP8_NF16
+#define MLA_FP8_NF16 3
+#endif
+
 template <int G, class SH = MlaShape>
 struct TransposedCfg {
     static_assert(G == 16 || G == 32, "query rows per CTA");
-    static constexpr int kThreads = 192;
+    // FP8 cache: + 4 converter warps (2 at G = 32, whose softmax needs the
+    // registers of a 256-thread block)
+    static constexpr int kConvThreads = SH::kFp8 ? ((G == 16) ? 128 : 64) : 0;
+    static constexpr int kThreads = 192 + kConvThreads;
     // pair slots [128 kv x 128 col]: an MLA tile needs 4 (+ a rope slot), an MHA
     // tile 2 (its K and its V)
-    static constexpr int NP = SH::kMha ? 6 : ((G == 16) ? 5 : 4);
-    static constexpr int NR = SH::kMha ? 1 : 2;   // rope slots (unused by MHA)
+    static constexpr int NP = SH::kMha ? 6 : SH::kFp8 ? ((G == 16) ? MLA_FP8_NP16 : 4) : ((G == 16) ? 5 : 4);
+    static constexpr int NR = (SH::kMha || SH::kFp8) ? 1 : 2;  // rope slots (unused by MHA)
+    static constexpr int NF = SH::kFp8 ? ((G == 16) ? MLA_FP8_NF16 : 4) : 0;  // FP8 staging slots
     static constexpr int kPairBytes = kTileKV * 128 * 2;     // 32 KB
     static constexpr int kChunkBytes = kTileKV * 128;        // 16 KB
+    static constexpr int kF8Bytes = kTileKV * kChunk;        // 8 KB: one chunk of E4M3 codes
     static constexpr int kQChunkBytes = G * 128;
     static constexpr int kPTBytes = kTileKV * G * 2;
     static constexpr int OFF_PAIR = 0;
     static constexpr int OFF_ROPE = OFF_PAIR + NP * kPairBytes;
     static constexpr int OFF_Q = OFF_ROPE + NR * kChunkBytes;
     static constexpr int OFF_PT = OFF_Q + SH::kQKChunks * kQChunkBytes;
-    static constexpr int OFF_RED = OFF_PT + kPTBytes;              // floats: [2][4][G] max, [4][G] sums
+    static constexpr int OFF_F8 = OFF_PT + kPTBytes;
+    static constexpr int OFF_RED = OFF_F8 + NF * kF8Bytes;          // floats: [2][4][G] max, [4][G] sums
     static constexpr int kRedFloats = 12 * G;
     static constexpr int OFF_BAR = OFF_RED + kRedFloats * 4;
     // barriers: q_full, q_empty, s_full, p_full, pv_done, drain, group_sync, pair_full[NP],
-    //           pair_empty[NP], rope_full[NR], rope_empty[NR]
-    static constexpr int kNumBars = 7 + 2 * NP + 2 * NR;
+    //           pair_empty[NP], rope_full[NR], rope_empty[NR], f8_full[NF], f8_empty[NF], q_ready
+    static constexpr int kNumBars = 7 + 2 * NP + 2 * NR + 2 * NF + (SH::kFp8 ? 1 : 0);
     static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
     static constexpr int kSmemBytes = OFF_MISC + 64 + 1024;  // + slack to align the base to 1024
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -126,8 +162,10 @@ struct TransposedCfg {
     // P^T swizzle: one row of G bf16 = 2G bytes (32 or 64)
     static constexpr ptx::Swizzle kPTSwz = (G == 16) ? ptx::Swizzle::B32 : ptx::Swizzle::B64;
     static constexpr uint32_t kPTAtom = 8 * 2 * G;  // 8 rows x row bytes
-    static constexpr uint32_t kIdescS = ptx::make_idesc_bf16(128, G, 0, 0);
-    static constexpr uint32_t kIdescPV = ptx::make_idesc_bf16(128, G, 1, 1);
+    static constexpr uint32_t kIdescS =
+        SH::kFp8 ? ptx::make_idesc_f16(128, G, 0, 0) : ptx::make_idesc_bf16(128, G, 0, 0);
+    static constexpr uint32_t kIdescPV =
+        SH::kFp8 ? ptx::make_idesc_f16(128, G, 1, 1) : ptx::make_idesc_bf16(128, G, 1, 1);
 };
 
 // Byte offset of 16-byte unit u of row r in a swizzled region whose rows are
@@ -137,6 +175,53 @@ __device__ __forceinline__ uint32_t swz_offset(uint32_t r, uint32_t u, uint32_t 
     const uint32_t addr = r * row_bytes + u * 16;
     const uint32_t mask = (row_bytes / 16) - 1;
     return addr ^ (((addr >> 7) & mask) << 4);
+}
+
+// Widening E4M3 codes to f16 with integer ALU operations (the hardware
+// e4m3x2 -> f16x2 conversion has a fraction of their throughput).  An E4M3
+// code s.eeee.mmm placed in an f16 as s.0eeee.mmm0000000 is, bit for bit,
+// the f16 of e4m3(code) * 2^-8: normals 2^(e-7)(1 + m/8) become 2^(e-15)(1 + m/8),
+// and subnormals (m/8) 2^-6 become the f16 subnormals (m/8) 2^-14.  The kernel
+// multiplies the 2^8 back into the score scale and the output scale.  The
+// NaN codes S.1111.111 read as +-480 * 2^-8: the cache must hold finite codes.
+constexpr float kF8Unscale = 256.f;
+
+// Four codes (byte k = column k) -> f16 pairs (columns 0, 1) and (2, 3), each
+// value e4m3(code) * 2^-8.
+__device__ __forceinline__ void e4m3x4_to_f16x4_div256(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+    const uint32_t w0 = __byte_perm(codes, 0u, 0x1404u);  // code 1 << 24 | code 0 << 8
+    const uint32_t w1 = __byte_perm(codes, 0u, 0x3424u);  // code 3 << 24 | code 2 << 8
+    lo = ((w0 & 0x7F007F00u) >> 1) | (w0 & 0x80008000u);
+    hi = ((w1 & 0x7F007F00u) >> 1) | (w1 & 0x80008000u);
+}
+
+// Eight bf16 -> eight f16 (round to nearest even; exact for |x| in [2^-17, 65504]).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        const __half2 h = __float22half2_rn(f);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Widens kv row r of one staged chunk: 64 E4M3 codes (64-byte rows, 64-byte
+// swizzle, as TMA wrote them) -> 64 f16 (each e4m3(code) * 2^-8) in the
+// 128-byte-swizzled K-major layout the MMA descriptors read (the layout TMA
+// gives a bf16 chunk).
+__device__ __forceinline__ void widen_chunk_row(const uint8_t* f8, uint8_t* dst, uint32_t r) {
+#pragma unroll
+    for (uint32_t u = 0; u < 4; ++u) {
+        const uint4 c = *reinterpret_cast<const uint4*>(f8 + swz_offset(r, u, 64));
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) e4m3x4_to_f16x4_div256(w[i], o[2 * i], o[2 * i + 1]);
+        *reinterpret_cast<uint4*>(dst + swz_offset(r, 2 * u, 128)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(dst + swz_offset(r, 2 * u + 1, 128)) = make_uint4(o[4], o[5], o[6], o[7]);
+    }
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -192,7 +277,7 @@ __device__ __forceinline__ int group_row(const MainArgs& a, int G, int g, int j)
 }
 
 template <int G, class SH = MlaShape>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(TransposedCfg<G, SH>::kThreads, 1)
     mla_decode_transposed_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                                  const __grid_constant__ CUtensorMap tm_v, const MainArgs args) {
     using C = TransposedCfg<G, SH>;
@@ -216,6 +301,10 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* pair_empty = pair_full + C::NP;
     uint64_t* rope_full = pair_empty + C::NP;
     uint64_t* rope_empty = rope_full + C::NR;
+    uint64_t* f8_full = rope_empty + C::NR;   // FP8 staging slot landed (TMA)
+    uint64_t* f8_empty = f8_full + C::NF;     // FP8 staging slot widened (converters)
+    uint64_t* q_ready = f8_empty + C::NF;     // FP8: Q narrowed to f16 in place
+    uint8_t* f8_smem = smem + C::OFF_F8;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     uint32_t* tmem_base_slot = misc + 0;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -238,14 +327,21 @@ __global__ void __launch_bounds__(192, 1)
         ptx::mbar_init(pv_done, 1);
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(group_sync, 128);
+        // FP8: the converter threads fill the operand slots, not TMA
+        const uint32_t fill_count = SH::kFp8 ? C::kConvThreads : 1;
         for (int i = 0; i < C::NP; ++i) {
-            ptx::mbar_init(pair_full + i, 1);
+            ptx::mbar_init(pair_full + i, fill_count);
             ptx::mbar_init(pair_empty + i, 1);
         }
         for (int i = 0; i < C::NR; ++i) {
-            ptx::mbar_init(rope_full + i, 1);
+            ptx::mbar_init(rope_full + i, fill_count);
             ptx::mbar_init(rope_empty + i, 1);
         }
+        for (int i = 0; i < C::NF; ++i) {
+            ptx::mbar_init(f8_full + i, 1);
+            ptx::mbar_init(f8_empty + i, C::kConvThreads);
+        }
+        if (SH::kFp8) ptx::mbar_init(q_ready, C::kConvThreads);
         *abort_flag = 0;
         ptx::fence_mbarrier_init();
     }
@@ -309,8 +405,31 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 4) {
         // ============================================================ TMA producer
         if (ptx::elect_one()) {
-            uint32_t pair_cnt = 0, rope_cnt = 0, piece_cnt = 0;
+            uint32_t pair_cnt = 0, rope_cnt = 0, piece_cnt = 0, f8_cnt = 0;
             int unit = 0;
+            // FP8 cache: L2 prefetch cursor `prefetch_tiles` tiles ahead of the
+            // staging loads, across piece boundaries (a tile's 9 chunk boxes,
+            // and the next piece's Q rows on entering it).  The staging ring
+            // holds few bytes, so without it the loads see HBM latency.
+            PieceWalker pf_walker = walker;
+            Piece pf_pc{};
+            bool pf_live = false, pf_started = false;
+            int pf_t = 0;
+            auto prefetch_next = [&](bool issue) {
+                if (!pf_live) return;
+                int r0 = pf_t * kTileKV;
+                if (r0 + kTileKV > pf_pc.L) r0 = pf_pc.L - kTileKV;
+                if (issue)
+                    for (int j = 0; j < kNumChunks; ++j) ptx::tma_prefetch_3d(&tm_kv, j * kChunk, r0, pf_pc.b);
+                if (++pf_t == pf_pc.tile_hi) {
+                    pf_live = pf_walker.next(pf_pc);
+                    if (pf_live) {
+                        pf_t = pf_pc.tile_lo;
+                        const int qrow = pf_pc.b * args.R + g * G;
+                        for (int c = 0; c < kNumChunks; ++c) ptx::tma_prefetch_2d(&tm_q, c * kChunk, qrow);
+                    }
+                }
+            };
             bool ok = true;
             // last armed phase per slot, for the drain on abort
             Piece pc;
@@ -354,6 +473,30 @@ __global__ void __launch_bounds__(192, 1)
                         }
                         continue;
                     }
+                    if constexpr (SH::kFp8) {
+                        if (!pf_started) {
+                            pf_started = true;
+                            pf_live = args.prefetch_tiles > 0 && pf_walker.next(pf_pc);
+                            pf_t = pf_live ? pf_pc.tile_lo : 0;
+                            prefetch_next(false);  // this tile: loaded now
+                            for (int i = 1; i < args.prefetch_tiles; ++i) prefetch_next(true);
+                        }
+                        prefetch_next(true);
+                        // the tile's 9 chunks of E4M3 codes (rope first, as the MMAs use them)
+                        for (int cc = 0; cc < kNumChunks; ++cc) {
+                            const int c = (cc == 0) ? kNumChunks - 1 : cc - 1;
+                            const uint32_t s = f8_cnt % C::NF;
+                            ok = ptx::mbar_wait_bounded(f8_empty + s, ((f8_cnt / C::NF) & 1) ^ 1, tmo);
+                            if (!ok) break;
+                            ptx::mbar_arrive_expect_tx(f8_full + s, C::kF8Bytes);
+                            if (!(blockIdx.x == 0 && unit == args.stall_unit))
+                                ptx::tma_load_3d(f8_smem + s * C::kF8Bytes, &tm_kv, f8_full + s, c * kChunk, row0,
+                                                 pc.b);
+                            ++unit;
+                            ++f8_cnt;
+                        }
+                        continue;
+                    }
                     {
                         const uint32_t s = rope_cnt % C::NR;
                         ok = ptx::mbar_wait_bounded(rope_empty + s, ((rope_cnt / C::NR) & 1) ^ 1, tmo);
@@ -389,8 +532,14 @@ __global__ void __launch_bounds__(192, 1)
             // Drain: every load this thread armed must have landed before the
             // CTA can exit (bounded; a load that was never issued -- the test
             // stall -- just runs the bound out).
-            if (piece_cnt > 0 || pair_cnt > 0) {
+            if (piece_cnt > 0 || pair_cnt > 0 || f8_cnt > 0) {
                 if (piece_cnt > 0) ptx::mbar_wait_bounded(q_full, (piece_cnt - 1) & 1, tmo);
+                if constexpr (SH::kFp8) {
+                    for (uint32_t i = 0; i < C::NF && i < f8_cnt; ++i) {
+                        const uint32_t use = f8_cnt - 1 - i;
+                        ptx::mbar_wait_bounded(f8_full + (use % C::NF), (use / C::NF) & 1, tmo);
+                    }
+                }
                 for (uint32_t i = 0; i < C::NP && i < pair_cnt; ++i) {
                     const uint32_t use = pair_cnt - 1 - i;  // the last use of slot use % NP
                     ptx::mbar_wait_bounded(pair_full + (use % C::NP), (use / C::NP) & 1, tmo);
@@ -416,7 +565,8 @@ __global__ void __launch_bounds__(192, 1)
                     const bool first = (t == pc.tile_lo);
                     const bool last = (t == pc.tile_hi - 1);
                     if (first) {
-                        ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
+                        // FP8: Q after the converters narrowed it to f16
+                        ok = ptx::mbar_wait_bounded(SH::kFp8 ? q_ready : q_full, piece_cnt & 1, tmo);
                         if (!ok) break;
                     }
                     if (SH::kMha) {
@@ -538,7 +688,7 @@ __global__ void __launch_bounds__(192, 1)
             ptx::mbar_wait_bounded(drain, 0, tmo);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 4) {
         // ============================================================ softmax + epilogue (warps 0-3)
         const int row_in_tile = warp * 32 + lane;            // TMEM lane = kv row (S^T) = dv row (O^T)
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
@@ -644,8 +794,13 @@ __global__ void __launch_bounds__(192, 1)
                     const float p1 = ex2_approx(x[j + 1] - m_ref[j + 1]);
                     l_part[j] += p0;
                     l_part[j + 1] += p1;
-                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    packed[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    if constexpr (SH::kFp8) {
+                        const __half2 h2 = __floats2half2_rn(p0, p1);
+                        packed[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    } else {
+                        const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        packed[j / 2] = *reinterpret_cast<const uint32_t*>(&h2);
+                    }
                 }
 #pragma unroll
                 for (int u = 0; u < (2 * G) / 16; ++u) {
@@ -687,7 +842,7 @@ __global__ void __launch_bounds__(192, 1)
                 float lj = redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j];
                 float c = 1.f;
                 if (sink_here) c = fold_sink(mj, lj, args.sinks[qr % args.H] * kLog2e);
-                fin[j] = c / lj;
+                fin[j] = c / lj * args.o_scale;
                 const float lse_nat = (mj + log2f(lj)) * 0.69314718055994530942f;
                 if (pc.slot < 0)
                     args.lse[static_cast<size_t>(pc.b) * args.R + qr] = lse_nat;
@@ -730,6 +885,65 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) {
             atomicOr(args.status, kStatusTimeout);
             *abort_flag = 1;
+        }
+    } else if (warp >= 6) {
+        // ============================================================ FP8 converters (warps 6..)
+        if constexpr (SH::kFp8) {
+            const uint32_t r = threadIdx.x - 192;  // first kv row of the tile this thread widens
+            uint32_t f8_cnt = 0, pair_cnt = 0, rope_cnt = 0, piece_cnt = 0;
+            bool ok = true;
+            Piece pc;
+            while (ok && walker.next(pc)) {
+                // this piece's Q rows: bf16 -> f16 in place (same element positions)
+                ok = ptx::mbar_wait_bounded(q_full, piece_cnt & 1, tmo);
+                if (!ok) break;
+                for (uint32_t i = r; i < kNumChunks * C::kQChunkBytes / 16; i += C::kConvThreads) {
+                    uint4* qp = reinterpret_cast<uint4*>(q_smem) + i;
+                    *qp = bf16x8_to_f16x8(*qp);
+                }
+                ptx::fence_proxy_async_smem();
+                ptx::mbar_arrive(q_ready);
+                for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
+                    for (int cc = 0; cc < kNumChunks; ++cc) {
+                        const int c = (cc == 0) ? kNumChunks - 1 : cc - 1;
+                        const uint32_t fs = f8_cnt % C::NF;
+                        ok = ptx::mbar_wait_bounded(f8_full + fs, (f8_cnt / C::NF) & 1, tmo);
+                        if (!ok) break;
+                        uint8_t* dst;
+                        if (c == kNumChunks - 1) {
+                            const uint32_t rs = rope_cnt % C::NR;
+                            ok = ptx::mbar_wait_bounded(rope_empty + rs, ((rope_cnt / C::NR) & 1) ^ 1, tmo);
+                            dst = rope_smem + rs * C::kChunkBytes;
+                        } else {
+                            const uint32_t ps = pair_cnt % C::NP;
+                            if ((c & 1) == 0)
+                                ok = ptx::mbar_wait_bounded(pair_empty + ps, ((pair_cnt / C::NP) & 1) ^ 1, tmo);
+                            dst = pair_smem + ps * C::kPairBytes + (c & 1) * C::kChunkBytes;
+                        }
+                        if (!ok) break;
+#pragma unroll
+                        for (uint32_t row = r; row < kTileKV; row += C::kConvThreads)
+                            widen_chunk_row(f8_smem + fs * C::kF8Bytes, dst, row);
+                        ptx::mbar_arrive(f8_empty + fs);  // codes read: the slot may be reloaded
+                        // an operand slot is complete: publish it to the tensor core
+                        if (c == kNumChunks - 1) {
+                            ptx::fence_proxy_async_smem();
+                            ptx::mbar_arrive(rope_full + rope_cnt % C::NR);
+                            ++rope_cnt;
+                        } else if (c & 1) {
+                            ptx::fence_proxy_async_smem();
+                            ptx::mbar_arrive(pair_full + pair_cnt % C::NP);
+                            ++pair_cnt;
+                        }
+                        ++f8_cnt;
+                    }
+                }
+                ++piece_cnt;
+            }
+            if (!ok) {
+                atomicOr(args.status, kStatusTimeout);
+                *abort_flag = 1;
+            }
         }
     }
 

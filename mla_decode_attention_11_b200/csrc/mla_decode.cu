@@ -145,6 +145,20 @@ bool encode_kv(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// FP8 cache: kv viewed as [B][L_max][576] bytes (E4M3 codes): a box of 128
+// rows x 64 codes, 64-byte swizzle (rows of 64 bytes)
+bool encode_kv_fp8(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int B) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(L_max),
+                                static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk),
+                                   static_cast<cuuint64_t>(mla::kDqk) * L_max};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), static_cast<cuuint32_t>(mla::kTileKV), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kv), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 extern "C" {
@@ -242,6 +256,23 @@ mla_status mla_decode_plan_batch_invariant(int32_t B, int32_t Sq, int32_t H, int
     return MLA_OK;
 }
 
+mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                               int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes) {
+    if (!plan) return MLA_ERR_INVALID_ARG;
+    mla_plan p;
+    const mla_status st =
+        mla_decode_plan_kernel(B, Sq, H, L_max, device, num_partitions_override, MLA_KERNEL_TRANSPOSED, &p, nullptr);
+    if (st != MLA_OK) return st;
+    p.kernel = MLA_KERNEL_FP8;
+    p.cta_threads = (p.group_rows == 16) ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kThreads
+                                         : mla::TransposedCfg<32, mla::MlaFp8Shape>::kThreads;
+    p.smem_bytes = (p.group_rows == 16) ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kSmemBytes
+                                        : mla::TransposedCfg<32, mla::MlaFp8Shape>::kSmemBytes;
+    *plan = p;
+    if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
+    return MLA_OK;
+}
+
 mla_status mla_decode_workspace_init(const mla_plan* plan, void* workspace, size_t workspace_bytes, void* stream) {
     if (!plan || !workspace) return MLA_ERR_INVALID_ARG;
     if (workspace_bytes < plan->workspace_bytes || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
@@ -256,12 +287,17 @@ mla_status mla_decode_workspace_init(const mla_plan* plan, void* workspace, size
 
 namespace {
 
+// kv_scale: null for a bf16 cache; for an FP8 cache (plan kind MLA_KERNEL_FP8)
+// the host address of its dequantization scale
 mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
                       float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
-                      size_t workspace_bytes, void* stream_, int phases) {
+                      size_t workspace_bytes, void* stream_, int phases, const float* kv_scale = nullptr) {
     if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
     if (!plan || !q || !kv || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
+    const bool fp8 = (plan->kernel == MLA_KERNEL_FP8);
+    if (fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;  // plan kind and entry point disagree
+    if (fp8 && !(std::isfinite(*kv_scale) && *kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
     const mla_plan& pl = *plan;
     const int R = pl.Sq * pl.H;
     if (pl.B < 1 || pl.Sq < 1 || pl.H < 1 || pl.L_max < 1 || pl.num_partitions < 1 || pl.num_groups < 1 ||
@@ -269,7 +305,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
         return MLA_ERR_INVALID_ARG;
     if (pl.l2_prefetch_tiles < 0 || pl.l2_prefetch_tiles > 16) return MLA_ERR_INVALID_ARG;
     if (pl.split_tiles < 0 || pl.split_tiles > (1 << 17)) return MLA_ERR_INVALID_ARG;
-    if (pl.kernel == MLA_KERNEL_TRANSPOSED) {
+    if (pl.kernel == MLA_KERNEL_TRANSPOSED || pl.kernel == MLA_KERNEL_FP8) {
         if (pl.group_rows != 16 && pl.group_rows != 32) return MLA_ERR_INVALID_ARG;
     } else if (pl.kernel == MLA_KERNEL_PAIR) {
         if (pl.group_rows != 128) return MLA_ERR_INVALID_ARG;
@@ -306,6 +342,10 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
             !encode_kv(enc, &tm_k, kv, pl.L_max, pl.B, 64) ||
             !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV))
             return MLA_ERR_CUDA;
+    } else if (fp8) {
+        if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, G) ||
+            !encode_kv_fp8(enc, &tm_kv, kv, pl.L_max, pl.B))
+            return MLA_ERR_CUDA;
     } else {
         if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, G) ||
             !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV))
@@ -321,7 +361,11 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     a.L_max = pl.L_max;
     a.P = pl.num_partitions;
     a.NG = pl.num_groups;
-    a.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * 1.4426950408889634074);
+    // an FP8 cache's scale multiplies every key (scores) and every value (output
+    // rows); the kernel's f16 operands hold the E4M3 values divided by 2^8
+    const double kvs = fp8 ? static_cast<double>(*kv_scale) * mla::kF8Unscale : 1.0;
+    a.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kvs * 1.4426950408889634074);
+    a.o_scale = static_cast<float>(kvs);
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
@@ -341,6 +385,9 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
         mla_status st;
         if (pl.kernel == MLA_KERNEL_PAIR)
             st = launch_pair(pl, tm_q, tm_k, tm_kv, a, stream);
+        else if (fp8)
+            st = (G == 16) ? launch_transposed<16, mla::MlaFp8Shape>(pl, tm_q, tm_kv, tm_kv, a, stream)
+                           : launch_transposed<32, mla::MlaFp8Shape>(pl, tm_q, tm_kv, tm_kv, a, stream);
         else
             st = (G == 16) ? launch_transposed<16>(pl, tm_q, tm_kv, tm_kv, a, stream)
                            : launch_transposed<32>(pl, tm_q, tm_kv, tm_kv, a, stream);
@@ -392,6 +439,21 @@ mla_status mla_decode_run_phase(const mla_plan* plan, const void* q, const void*
     if (phase != 1 && phase != 2) return MLA_ERR_INVALID_ARG;
     return run_phases(plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, workspace, workspace_bytes, stream,
                       phase);
+}
+
+mla_status mla_decode_run_fp8(const mla_plan* plan, const void* q, const void* kv_fp8, float kv_scale,
+                              const int32_t* seqlens, float softmax_scale, const float* sinks, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    return run_phases(plan, q, kv_fp8, seqlens, softmax_scale, sinks, out, lse, workspace, workspace_bytes, stream, 3,
+                      &kv_scale);
+}
+
+mla_status mla_decode_run_fp8_phase(const mla_plan* plan, const void* q, const void* kv_fp8, float kv_scale,
+                                    const int32_t* seqlens, float softmax_scale, void* out, float* lse,
+                                    void* workspace, size_t workspace_bytes, void* stream, int32_t phase) {
+    if (phase != 1 && phase != 2) return MLA_ERR_INVALID_ARG;
+    return run_phases(plan, q, kv_fp8, seqlens, softmax_scale, nullptr, out, lse, workspace, workspace_bytes, stream,
+                      phase, &kv_scale);
 }
 
 mla_status mla_decode_check(const mla_plan* plan, void* workspace, void* stream) {
@@ -650,6 +712,7 @@ mla_status mha_run_phases(const mla_plan* plan, const void* q, const void* k, co
     a.split_tiles = pl.split_tiles;
     a.Sq = pl.Sq;
     a.Hkv = pl.Hkv;
+    a.o_scale = 1.f;
     if (phases & 1) {
         const mla_status st = (G == 16) ? launch_transposed<16, mla::MhaShape>(pl, tm_q, tm_k, tm_v, a, stream)
                                         : launch_transposed<32, mla::MhaShape>(pl, tm_q, tm_k, tm_v, a, stream);

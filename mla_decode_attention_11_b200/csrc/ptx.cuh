@@ -353,8 +353,17 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and f32 D.
+// Instruction descriptors for kind::f16 with f32 D: A and B both f16 (format
+// code 0) or both bf16 (format code 1).
 // a_mn / b_mn: 1 = operand stored MN-major (M resp. N contiguous), 0 = K-major.
+__host__ __device__ constexpr uint32_t make_idesc_f16(uint32_t M, uint32_t N, uint32_t a_mn, uint32_t b_mn) {
+    return (1u << 4)            // D format: f32
+           | (a_mn << 15)       // A major
+           | (b_mn << 16)       // B major
+           | ((N >> 3) << 17)   // N / 8
+           | ((M >> 4) << 24);  // M / 16
+}
+
 __host__ __device__ constexpr uint32_t make_idesc_bf16(uint32_t M, uint32_t N, uint32_t a_mn, uint32_t b_mn) {
     return (1u << 4)            // D format: f32
            | (1u << 7)          // A format: bf16

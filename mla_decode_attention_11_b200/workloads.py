@@ -55,6 +55,12 @@ class Workload:
         rows = self.B * self.Sq * self.H
         return int(sl.to(torch.int64).sum()) * D_QK * 2 + rows * (D_QK * 2 + D_V * 2 + 4) + self.B * 4
 
+    def algorithmic_bytes_fp8(self, lengths: Optional[torch.Tensor] = None) -> int:
+        """As algorithmic_bytes with the cache held as one-byte E4M3 codes."""
+        sl = self.lengths() if lengths is None else lengths
+        rows = self.B * self.Sq * self.H
+        return int(sl.to(torch.int64).sum()) * D_QK + rows * (D_QK * 2 + D_V * 2 + 4) + self.B * 4
+
     def algorithmic_flops(self, lengths: Optional[torch.Tensor] = None) -> int:
         """2*(576+512) flops per (query row, key): QK^T and PV, exps not counted."""
         sl = self.lengths() if lengths is None else lengths
@@ -101,6 +107,26 @@ def generate(w: Workload, tail_fill: float = float("nan"), lengths: Optional[tor
         if Lb < w.L:
             kv[b, Lb:] = tail_fill
     return q, kv, sl
+
+
+E4M3_MAX = 448.0
+E4M3_NAN_CODE = 0x7F
+
+
+def generate_fp8(w: Workload, lengths: Optional[torch.Tensor] = None):
+    """The same inputs with the cache quantised to E4M3 codes: (q [B,Sq,H,576]
+    bf16, codes [B,L_max,576] uint8, kv_scale, seqlens [B]).  kv_scale =
+    max|kv| / 448 over the used rows (per-tensor amax scaling, as an fp32
+    value); each bf16 value is divided by it and rounded to the nearest E4M3
+    code by torch's own conversion.  Rows at or past a length hold the NaN
+    code (never a value of the used rows), so a read past a length shows."""
+    q, kv, sl = generate(w, tail_fill=0.0, lengths=lengths)
+    amax = float(kv.float().abs().max())
+    kv_scale = float(torch.tensor(max(amax, 1e-30) / E4M3_MAX, dtype=torch.float32).item())
+    codes = (kv.float() / kv_scale).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+    for b in range(w.B):
+        codes[b, int(sl[b]):] = E4M3_NAN_CODE
+    return q, codes.contiguous(), kv_scale, sl
 
 
 def small_variant(w: Workload, B: Optional[int] = None, L: Optional[int] = None,

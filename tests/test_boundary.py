@@ -122,3 +122,42 @@ def test_batch_invariant_plan_without_gpu():
     assert b.split_tiles == 0
     with pytest.raises(M.MlaError):
         M.mla_decode_plan_batch_invariant(64, 1, 128, 8192, device=-1, split_tiles=-1)
+
+
+def test_fp8_plan_without_gpu():
+    p = M.mla_decode_plan_fp8(132, 1, 16, 16384, device=-1)
+    assert p.kernel == M.MLA_KERNEL_FP8 and p.group_rows == 16 and p.cta_threads == 320
+    assert p.num_partitions == 148 and p.smem_bytes <= 232448
+    p = M.mla_decode_plan_fp8(64, 1, 128, 8192, device=-1)
+    assert p.kernel == M.MLA_KERNEL_FP8 and p.group_rows == 32 and p.num_groups == 4 and p.cta_threads == 256
+    assert p.workspace_bytes == M.mla_decode_plan(64, 1, 128, 8192, device=-1,
+                                                  kernel=M.MLA_KERNEL_TRANSPOSED).workspace_bytes
+    with pytest.raises(M.MlaError) as e:
+        M.mla_decode_plan_fp8(64, 1, 24, 8192, device=-1)
+    assert e.value.code == 3
+
+
+def test_fp8_run_rejects_without_launching(lib):
+    """A plan of the other kind, a kv_scale that is not finite and positive,
+    null pointers and misalignment are refused on the host."""
+    f8 = M.mla_decode_plan_fp8(2, 1, 16, 256, device=-1)
+    bf = M.mla_decode_plan(2, 1, 16, 256, device=-1)
+    run8 = lib.mla_decode_run_fp8
+    ok_scale, sc = ctypes.c_float(0.01), ctypes.c_float(0.04)
+    rc = run8(ctypes.byref(bf), 16, 16, ok_scale, 16, sc, None, 16, 16, 256, bf.workspace_bytes, None)
+    assert rc == 1
+    for bad in (0.0, -0.5, float("nan"), float("inf")):
+        rc = run8(ctypes.byref(f8), 16, 16, ctypes.c_float(bad), 16, sc, None, 16, 16, 256, f8.workspace_bytes, None)
+        assert rc == 1
+    rc = run8(ctypes.byref(f8), 16, None, ok_scale, 16, sc, None, 16, 16, 256, f8.workspace_bytes, None)
+    assert rc == 1
+    rc = run8(ctypes.byref(f8), 16, 16 + 4, ok_scale, 16, sc, None, 16, 16, 256, f8.workspace_bytes, None)
+    assert rc == 2
+    rc = run8(ctypes.byref(f8), 16, 16, ok_scale, 16, sc, None, 16, 16, 256, f8.workspace_bytes - 1, None)
+    assert rc == 6
+    # the bf16 entry points refuse an FP8 plan
+    rc = lib.mla_decode_run(ctypes.byref(f8), 16, 16, 16, sc, 16, 16, 256, f8.workspace_bytes, None)
+    assert rc == 1
+    rc = lib.mla_decode_run_fp8_phase(ctypes.byref(f8), 16, 16, ok_scale, 16, sc, 16, 16, 256, f8.workspace_bytes,
+                                      None, 3)
+    assert rc == 1
