@@ -39,6 +39,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "ptx.cuh"
@@ -177,13 +178,17 @@ __device__ __forceinline__ uint32_t swz_offset(uint32_t r, uint32_t u, uint32_t 
     return addr ^ (((addr >> 7) & mask) << 4);
 }
 
-// Widening E4M3 codes to f16 with integer ALU operations (the hardware
-// e4m3x2 -> f16x2 conversion has a fraction of their throughput).  An E4M3
-// code s.eeee.mmm placed in an f16 as s.0eeee.mmm0000000 is, bit for bit,
-// the f16 of e4m3(code) * 2^-8: normals 2^(e-7)(1 + m/8) become 2^(e-15)(1 + m/8),
-// and subnormals (m/8) 2^-6 become the f16 subnormals (m/8) 2^-14.  The kernel
-// multiplies the 2^8 back into the score scale and the output scale.  The
-// NaN codes S.1111.111 read as +-480 * 2^-8: the cache must hold finite codes.
+// Widening E4M3 codes to f16 values e4m3(code) * 2^-8 (exact; the kernel
+// multiplies the 2^8 back into the score scale and the output scale).  Two
+// routes, used for alternate words of a chunk because each alone saturates
+// its pipe (measured: half and half is ~10% faster than either):
+//  - integer ALU: a code s.eeee.mmm placed in an f16 as s.0eeee.mmm0000000 is,
+//    bit for bit, the f16 of e4m3(code) * 2^-8 (normals 2^(e-7)(1 + m/8) become
+//    2^(e-15)(1 + m/8), subnormals (m/8) 2^-6 become the f16 subnormals
+//    (m/8) 2^-14);
+//  - the hardware e4m3x2 -> f16x2 conversion, then an exact f16 multiply by 2^-8.
+// The cache must hold finite codes: the integer route reads the NaN codes
+// S.1111.111 as +-480 * 2^-8.
 constexpr float kF8Unscale = 256.f;
 
 // Four codes (byte k = column k) -> f16 pairs (columns 0, 1) and (2, 3), each
@@ -193,6 +198,17 @@ __device__ __forceinline__ void e4m3x4_to_f16x4_div256(uint32_t codes, uint32_t&
     const uint32_t w1 = __byte_perm(codes, 0u, 0x3424u);  // code 3 << 24 | code 2 << 8
     lo = ((w0 & 0x7F007F00u) >> 1) | (w0 & 0x80008000u);
     hi = ((w1 & 0x7F007F00u) >> 1) | (w1 & 0x80008000u);
+}
+
+// The same four values through the conversion unit.
+__device__ __forceinline__ void e4m3x4_to_f16x4_div256_cvt(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+    const __half2 k = __float2half2_rn(0.00390625f);  // 2^-8
+    __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xFFFFu), __NV_E4M3);
+    __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes >> 16), __NV_E4M3);
+    const __half2 ha = __hmul2(*reinterpret_cast<const __half2*>(&a), k);
+    const __half2 hb = __hmul2(*reinterpret_cast<const __half2*>(&b), k);
+    lo = *reinterpret_cast<const uint32_t*>(&ha);
+    hi = *reinterpret_cast<const uint32_t*>(&hb);
 }
 
 // Eight bf16 -> eight f16 (round to nearest even; exact for |x| in [2^-17, 65504]).
@@ -218,7 +234,12 @@ __device__ __forceinline__ void widen_chunk_row(const uint8_t* f8, uint8_t* dst,
         const uint32_t w[4] = {c.x, c.y, c.z, c.w};
         uint32_t o[8];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) e4m3x4_to_f16x4_div256(w[i], o[2 * i], o[2 * i + 1]);
+        for (int i = 0; i < 4; ++i) {
+            if (i < 2)
+                e4m3x4_to_f16x4_div256_cvt(w[i], o[2 * i], o[2 * i + 1]);
+            else
+                e4m3x4_to_f16x4_div256(w[i], o[2 * i], o[2 * i + 1]);
+        }
         *reinterpret_cast<uint4*>(dst + swz_offset(r, 2 * u, 128)) = make_uint4(o[0], o[1], o[2], o[3]);
         *reinterpret_cast<uint4*>(dst + swz_offset(r, 2 * u + 1, 128)) = make_uint4(o[4], o[5], o[6], o[7]);
     }
