@@ -37,6 +37,22 @@ METRIC = "MLA decode TFLOP/s + HBM GB/s at B=64,H=128,L=8192; fraction of roofli
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest of every rank's x (a multi-GPU job takes as long as its
+    slowest rank); x itself when dist is None (one process)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank
+    (independent replicas, weak scaling) in ms milliseconds, the max over ranks."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -251,10 +267,7 @@ def run_ours(args, w: W.Workload):
         dist.barrier()
     t_ms = e0.elapsed_time(e1) / args.steps
     M.mla_decode_check(plan, ws, stream=stream)
-    if dist:
-        t = torch.tensor([t_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_ms = float(t.item())
+    t_ms = max_over_ranks(t_ms, dist, dev)
 
     # ---- per-kernel breakdown: the same launches, each kernel alone, back to
     # back in a graph (phase 1 = main kernel, phase 2 = split-KV combine)
@@ -295,10 +308,7 @@ def run_ours(args, w: W.Workload):
         f1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = f0.elapsed_time(f1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     h2d = q.numel() * 2 + kv.numel() * 2 + sl.numel() * 4
     d2h = outh.numel() * 2 + lseh.numel() * 4
     M.mla_decode_check(plan, ws, stream=stream)
@@ -306,8 +316,8 @@ def run_ours(args, w: W.Workload):
     flops = w.algorithmic_flops(sl)
     nbytes = w.algorithmic_bytes(sl)
     peaks, peak_src = load_peaks()
-    value = world * flops / (t_ms * 1e-3) / 1e12
-    hbm_gbs = world * nbytes / (t_ms * 1e-3) / 1e9
+    value = whole_job_rate(world, flops, t_ms) / 1e12
+    hbm_gbs = whole_job_rate(world, nbytes, t_ms) / 1e9
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     ai = flops / nbytes
     bound = "hbm" if ai < ridge else "tensor"
@@ -354,7 +364,7 @@ def run_ours(args, w: W.Workload):
                          "tensor_tflops": flops / (main_avg * 1e-3) / 1e12,
                          "tensor_frac": flops / (main_avg * 1e-3) / 1e12 / peaks["bf16_tflops"],
                          "step_roofline_frac": roof_time_ms / t_ms, "traffic_note": traffic_note},
-            "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_rate(world, flops, e2e_ms) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
