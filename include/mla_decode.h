@@ -63,8 +63,10 @@ enum {
     MLA_KERNEL_TRANSPOSED = 1, /* S^T = K Q^T per CTA, kv rows on the 128 TMEM lanes (any H*Sq) */
     MLA_KERNEL_PAIR = 2,       /* CTA pair, 64 query rows per CTA, cta_group::2 MMAs (H*Sq % 128 == 0) */
     MLA_KERNEL_MHA = 3,        /* MHA decode (mha_decode_plan): the transposed kernel over 128-wide K, V */
-    MLA_KERNEL_FP8 = 4         /* MLA decode over an FP8 cache (mla_decode_plan_fp8): the transposed kernel
+    MLA_KERNEL_FP8 = 4,        /* MLA decode over an FP8 cache (mla_decode_plan_fp8): the transposed kernel
                                   with E4M3 chunks widened to f16 in shared memory */
+    MLA_KERNEL_FP8_MMA = 5     /* MLA decode over an FP8 cache with the codes as kind::f8f6f4 MMA operands
+                                  (mla_decode_plan_fp8_kernel); experimental, see there */
 };
 
 /*
@@ -350,6 +352,22 @@ mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void*
  */
 mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
                                int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
+
+/*
+ * mla_decode_plan_fp8_kernel -- mla_decode_plan_fp8 with an explicit kernel:
+ *   kernel  0 or MLA_KERNEL_FP8: the widening kernel (what mla_decode_plan_fp8 picks);
+ *           MLA_KERNEL_FP8_MMA: EXPERIMENTAL, not yet validated on a GPU -- the
+ *           codes are the operands of kind::f8f6f4 MMAs and q and P are carried
+ *           as sums of E4M3 terms (q: three terms of a power-of-two-scaled row,
+ *           about 12 significant bits; P: two terms, about 8), so its results
+ *           differ from the exact-operand path by those truncations.
+ *           Anything else: MLA_ERR_INVALID_ARG.
+ * Other arguments and return codes as mla_decode_plan_fp8; the plan runs
+ * through mla_decode_run_fp8.
+ */
+mla_status mla_decode_plan_fp8_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                                      int32_t num_partitions_override, int32_t kernel, mla_plan* plan,
+                                      size_t* workspace_bytes);
 
 /*
  * mla_decode_run_fp8 -- enqueue one MLA decode over an FP8 cache on `stream`.

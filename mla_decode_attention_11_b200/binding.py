@@ -34,6 +34,7 @@ MLA_KERNEL_TRANSPOSED = 1
 MLA_KERNEL_PAIR = 2
 MLA_KERNEL_MHA = 3
 MLA_KERNEL_FP8 = 4
+MLA_KERNEL_FP8_MMA = 5
 MHA_D = 128
 MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
@@ -41,7 +42,8 @@ EXPORTED_SYMBOLS = ("mla_decode_plan", "mla_decode_plan_kernel", "mla_decode_pla
                     "mla_decode_check", "mla_decode_run_noalloc", "mla_decode_run_sinks",
                     "mla_status_string", "mla_decode_abi_version", "mla_decode_set_debug",
                     "mha_decode_plan", "mha_decode_run", "mha_decode_run_phase",
-                    "mla_decode_plan_fp8", "mla_decode_run_fp8", "mla_decode_run_fp8_phase")
+                    "mla_decode_plan_fp8", "mla_decode_plan_fp8_kernel", "mla_decode_run_fp8",
+                    "mla_decode_run_fp8_phase")
 
 
 class MlaError(RuntimeError):
@@ -120,6 +122,9 @@ def load_library(build_if_missing: bool = True):
         lib.mla_decode_plan_fp8.restype = c_i32
         lib.mla_decode_plan_fp8.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, ctypes.POINTER(mla_plan),
                                             ctypes.POINTER(c_sz)]
+        lib.mla_decode_plan_fp8_kernel.restype = c_i32
+        lib.mla_decode_plan_fp8_kernel.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                                   ctypes.POINTER(mla_plan), ctypes.POINTER(c_sz)]
         lib.mla_decode_run_fp8.restype = c_i32
         lib.mla_decode_run_fp8.argtypes = [ctypes.POINTER(mla_plan), c_vp, c_vp, c_f, c_vp, c_f, c_vp, c_vp, c_vp,
                                            c_vp, c_sz, c_vp]
@@ -401,17 +406,19 @@ def mha_decode_run_phase(plan: mla_plan, q, k, v, seqlens, softmax_scale: float,
 # ---------------------------------------------------------------- FP8 latent cache
 
 def mla_decode_plan_fp8(B: int, Sq: int, H: int, L_max: int, device: Optional[int] = None,
-                        num_partitions: int = 0) -> mla_plan:
+                        num_partitions: int = 0, kernel: int = 0) -> mla_plan:
     """A plan for a cache of E4M3 codes (mla_decode_plan_fp8): the transposed
-    kernel with FP8 staging, for every head count."""
+    kernel with FP8 staging, for every head count.  kernel = MLA_KERNEL_FP8_MMA
+    selects the experimental FP8-operand kernel (mla_decode_plan_fp8_kernel)."""
     if device is None:
         device = torch.cuda.current_device()
     p = mla_plan()
     ws = ctypes.c_size_t(0)
-    rc = load_library().mla_decode_plan_fp8(int(B), int(Sq), int(H), int(L_max), int(device), int(num_partitions),
-                                            ctypes.byref(p), ctypes.byref(ws))
+    rc = load_library().mla_decode_plan_fp8_kernel(int(B), int(Sq), int(H), int(L_max), int(device),
+                                                   int(num_partitions), int(kernel), ctypes.byref(p),
+                                                   ctypes.byref(ws))
     if rc != MLA_OK:
-        raise MlaError(rc, "mla_decode_plan_fp8")
+        raise MlaError(rc, "mla_decode_plan_fp8_kernel")
     return p
 
 

@@ -69,6 +69,7 @@ struct MainArgs {
     int Sq;              // query tokens per sequence
     int Hkv;             // MHA: kv heads (query head h reads kv head h / (H / Hkv)); MLA: 1
     float o_scale;       // factor on every output row: the FP8 cache's kv_scale, else 1
+    const __nv_bfloat16* q;  // [B*R, 576] query rows (read directly by the FP8-operand kernel)
 };
 
 // The two attention shapes the transposed kernel serves.

@@ -20,6 +20,7 @@
 #include "kernel_combine.cuh"
 #include "kernel_pair.cuh"
 #include "kernel_transposed.cuh"
+#include "kernel_fp8mma.cuh"
 
 namespace {
 
@@ -81,6 +82,18 @@ mla_status launch_transposed(const mla_plan& plan, const CUtensorMap& tm_q, cons
         return MLA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(plan.num_partitions * plan.num_groups));
     kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_q, tm_kv, tm_v, args);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+template <int G>
+mla_status launch_fp8mma(const mla_plan& plan, const CUtensorMap& tm_kv, const mla::MainArgs& args,
+                         cudaStream_t stream) {
+    using C = mla::Fp8MmaCfg<G>;
+    auto kern = mla::mla_decode_fp8mma_kernel<G>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(plan.num_partitions * plan.num_groups));
+    kern<<<grid, C::kThreads, C::kSmemBytes, stream>>>(tm_kv, args);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -258,16 +271,30 @@ mla_status mla_decode_plan_batch_invariant(int32_t B, int32_t Sq, int32_t H, int
 
 mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
                                int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes) {
+    return mla_decode_plan_fp8_kernel(B, Sq, H, L_max, device, num_partitions_override, 0, plan, workspace_bytes);
+}
+
+mla_status mla_decode_plan_fp8_kernel(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
+                                      int32_t num_partitions_override, int32_t kernel, mla_plan* plan,
+                                      size_t* workspace_bytes) {
     if (!plan) return MLA_ERR_INVALID_ARG;
+    if (kernel == 0) kernel = MLA_KERNEL_FP8;
+    if (kernel != MLA_KERNEL_FP8 && kernel != MLA_KERNEL_FP8_MMA) return MLA_ERR_INVALID_ARG;
     mla_plan p;
     const mla_status st =
         mla_decode_plan_kernel(B, Sq, H, L_max, device, num_partitions_override, MLA_KERNEL_TRANSPOSED, &p, nullptr);
     if (st != MLA_OK) return st;
-    p.kernel = MLA_KERNEL_FP8;
-    p.cta_threads = (p.group_rows == 16) ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kThreads
-                                         : mla::TransposedCfg<32, mla::MlaFp8Shape>::kThreads;
-    p.smem_bytes = (p.group_rows == 16) ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kSmemBytes
-                                        : mla::TransposedCfg<32, mla::MlaFp8Shape>::kSmemBytes;
+    p.kernel = kernel;
+    const bool g16 = (p.group_rows == 16);
+    if (kernel == MLA_KERNEL_FP8) {
+        p.cta_threads = g16 ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kThreads
+                            : mla::TransposedCfg<32, mla::MlaFp8Shape>::kThreads;
+        p.smem_bytes = g16 ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kSmemBytes
+                           : mla::TransposedCfg<32, mla::MlaFp8Shape>::kSmemBytes;
+    } else {
+        p.cta_threads = mla::Fp8MmaCfg<16>::kThreads;
+        p.smem_bytes = g16 ? mla::Fp8MmaCfg<16>::kSmemBytes : mla::Fp8MmaCfg<32>::kSmemBytes;
+    }
     *plan = p;
     if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
     return MLA_OK;
@@ -295,7 +322,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
     if (!plan || !q || !kv || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
-    const bool fp8 = (plan->kernel == MLA_KERNEL_FP8);
+    const bool fp8 = (plan->kernel == MLA_KERNEL_FP8 || plan->kernel == MLA_KERNEL_FP8_MMA);
     if (fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;  // plan kind and entry point disagree
     if (fp8 && !(std::isfinite(*kv_scale) && *kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
     const mla_plan& pl = *plan;
@@ -305,7 +332,7 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
         return MLA_ERR_INVALID_ARG;
     if (pl.l2_prefetch_tiles < 0 || pl.l2_prefetch_tiles > 16) return MLA_ERR_INVALID_ARG;
     if (pl.split_tiles < 0 || pl.split_tiles > (1 << 17)) return MLA_ERR_INVALID_ARG;
-    if (pl.kernel == MLA_KERNEL_TRANSPOSED || pl.kernel == MLA_KERNEL_FP8) {
+    if (pl.kernel == MLA_KERNEL_TRANSPOSED || fp8) {
         if (pl.group_rows != 16 && pl.group_rows != 32) return MLA_ERR_INVALID_ARG;
     } else if (pl.kernel == MLA_KERNEL_PAIR) {
         if (pl.group_rows != 128) return MLA_ERR_INVALID_ARG;
@@ -362,10 +389,14 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     a.P = pl.num_partitions;
     a.NG = pl.num_groups;
     // an FP8 cache's scale multiplies every key (scores) and every value (output
-    // rows); the kernel's f16 operands hold the E4M3 values divided by 2^8
-    const double kvs = fp8 ? static_cast<double>(*kv_scale) * mla::kF8Unscale : 1.0;
+    // rows); the widening kernel's f16 operands hold the E4M3 values divided by
+    // 2^8, the FP8-operand kernel multiplies the codes themselves
+    const double kvs = !fp8 ? 1.0
+                            : static_cast<double>(*kv_scale) *
+                                  (pl.kernel == MLA_KERNEL_FP8 ? static_cast<double>(mla::kF8Unscale) : 1.0);
     a.scale_log2 = static_cast<float>(static_cast<double>(softmax_scale) * kvs * 1.4426950408889634074);
     a.o_scale = static_cast<float>(kvs);
+    a.q = static_cast<const __nv_bfloat16*>(q);
     a.out = static_cast<__nv_bfloat16*>(out);
     a.lse = lse;
     a.part_o = reinterpret_cast<float*>(ws + lay.part_o_off);
@@ -385,6 +416,8 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
         mla_status st;
         if (pl.kernel == MLA_KERNEL_PAIR)
             st = launch_pair(pl, tm_q, tm_k, tm_kv, a, stream);
+        else if (pl.kernel == MLA_KERNEL_FP8_MMA)
+            st = (G == 16) ? launch_fp8mma<16>(pl, tm_kv, a, stream) : launch_fp8mma<32>(pl, tm_kv, a, stream);
         else if (fp8)
             st = (G == 16) ? launch_transposed<16, mla::MlaFp8Shape>(pl, tm_q, tm_kv, tm_kv, a, stream)
                            : launch_transposed<32, mla::MlaFp8Shape>(pl, tm_q, tm_kv, tm_kv, a, stream);
@@ -713,6 +746,7 @@ mla_status mha_run_phases(const mla_plan* plan, const void* q, const void* k, co
     a.Sq = pl.Sq;
     a.Hkv = pl.Hkv;
     a.o_scale = 1.f;
+    a.q = static_cast<const __nv_bfloat16*>(q);
     if (phases & 1) {
         const mla_status st = (G == 16) ? launch_transposed<16, mla::MhaShape>(pl, tm_q, tm_k, tm_v, a, stream)
                                         : launch_transposed<32, mla::MhaShape>(pl, tm_q, tm_k, tm_v, a, stream);

@@ -161,3 +161,16 @@ def test_fp8_run_rejects_without_launching(lib):
     rc = lib.mla_decode_run_fp8_phase(ctypes.byref(f8), 16, 16, ok_scale, 16, sc, 16, 16, 256, f8.workspace_bytes,
                                       None, 3)
     assert rc == 1
+
+
+def test_fp8_operand_kernel_plan_without_gpu():
+    """The experimental FP8-operand kernel is only ever chosen explicitly."""
+    assert M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1).kernel == M.MLA_KERNEL_FP8
+    for H, G in ((16, 16), (128, 32)):
+        p = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8_MMA)
+        assert p.kernel == M.MLA_KERNEL_FP8_MMA and p.group_rows == G and p.cta_threads == 192
+        assert p.smem_bytes <= 232448
+    for bad in (1, 2, 3, 6):
+        with pytest.raises(M.MlaError) as e:
+            M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1, kernel=bad)
+        assert e.value.code == 1
