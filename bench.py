@@ -497,7 +497,8 @@ def run_fp8(args, w: W.Workload):
     torch.cuda.set_device(dev)
     q, codes, ks, sl = W.generate_fp8(w)
     qd, cd, sld = q.to(dev), codes.to(dev), sl.to(dev)
-    plan = M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=0)
+    kernel = M.MLA_KERNEL_FP8_MMA if args.fp8_kernel == "operands" else M.MLA_KERNEL_FP8
+    plan = M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=0, kernel=kernel)
     ws = M.alloc_workspace(plan, device=dev)
     M.mla_decode_workspace_init(plan, ws)
     out = torch.empty((w.B, w.Sq, w.H, W.D_V), dtype=torch.bfloat16, device=dev)
@@ -587,16 +588,20 @@ def run_fp8(args, w: W.Workload):
         "metric": METRIC + " (FP8 latent cache)",
         "value": flops / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 cache, f16 MMA", "data": "synthetic",
+        "vs_baseline": None,
+        "dtype": "e4m3 cache, e4m3 MMA" if kernel == M.MLA_KERNEL_FP8_MMA else "e4m3 cache, f16 MMA",
+        "data": "synthetic",
         "config": {"workload": workload_desc(w) + f"; cache quantised to E4M3, kv_scale = amax/448 = {ks:.6g}",
-                   "global_batch": w.B, "seq_len": w.L, "parallelism": "single GPU", "kernel": "transposed (FP8)",
+                   "global_batch": w.B, "seq_len": w.L, "parallelism": "single GPU",
+                   "kernel": "FP8 operands (kind::f8f6f4)" if kernel == M.MLA_KERNEL_FP8_MMA else "transposed (FP8)",
                    "group_rows": plan.group_rows, "partitions": plan.num_partitions,
                    "l2": "inputs larger than L2 (kv %.0f MB > 126 MB), no flush" % (codes.numel() / 1e6)},
         "hbm_gbs": nbytes / (t_ms * 1e-3) / 1e9,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                      "traffic_note": traffic_note,
-                     "kernel": "mla_decode_transposed_kernel<G, MlaFp8Shape>", "kernel_ms": main_ms,
+                     "kernel": ("mla_decode_fp8mma_kernel<G>" if kernel == M.MLA_KERNEL_FP8_MMA
+                                else "mla_decode_transposed_kernel<G, MlaFp8Shape>"), "kernel_ms": main_ms,
                      "combine_ms": comb_ms, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
                      "hbm_frac": nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "step_roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
@@ -625,6 +630,9 @@ def main():
                     help="time the attention-sink entry point (per-head sink logits) on the same workload")
     ap.add_argument("--fp8", action="store_true",
                     help="the same MLA workload over an FP8 (E4M3) latent cache (mla_decode_run_fp8)")
+    ap.add_argument("--fp8-kernel", choices=["widen", "operands"], default="widen",
+                    help="FP8 cache kernel: codes widened to f16 (default) or the experimental "
+                         "kind::f8f6f4 operand kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
