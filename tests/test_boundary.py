@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from mla_decode_attention_11_b200 import build as B
 from mla_decode_attention_11_b200 import binding as M
@@ -174,3 +175,23 @@ def test_fp8_operand_kernel_plan_without_gpu():
         with pytest.raises(M.MlaError) as e:
             M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1, kernel=bad)
         assert e.value.code == 1
+
+
+def test_fp8_input_generator():
+    """generate_fp8: kv_scale = max|kv| / 448 over the used rows (fp32), codes
+    are torch's E4M3 rounding of kv / kv_scale, and rows past a length hold
+    the NaN code; q and lengths are those of the bf16 generator."""
+    from mla_decode_attention_11_b200 import workloads as W
+    w = W.custom(B=3, Sq=1, H=16, L=300, L_lo=10, seed=77)
+    q, codes, ks, sl = W.generate_fp8(w)
+    q0, kv, sl0 = W.generate(w, tail_fill=0.0)
+    assert torch.equal(q, q0) and torch.equal(sl, sl0) and codes.dtype == torch.uint8
+    used = torch.cat([kv[b, :int(sl[b])] for b in range(w.B)]).float()
+    assert ks == float(torch.tensor(float(used.abs().max()) / 448.0, dtype=torch.float32))
+    for b in range(w.B):
+        L = int(sl[b])
+        vals = codes[b, :L].view(torch.float8_e4m3fn).float()
+        assert torch.isfinite(vals).all() and vals.abs().max() <= 448
+        ref = (kv[b, :L].float() / ks).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        assert torch.equal(codes[b, :L], ref)
+        assert (codes[b, L:] == W.E4M3_NAN_CODE).all()
