@@ -195,3 +195,43 @@ def test_fp8_input_generator():
         ref = (kv[b, :L].float() / ks).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
         assert torch.equal(codes[b, :L], ref)
         assert (codes[b, L:] == W.E4M3_NAN_CODE).all()
+
+
+def test_mha_plan_without_gpu():
+    p = M.mha_decode_plan(64, 1, 32, 8, 8192, device=-1)
+    assert p.kernel == M.MLA_KERNEL_MHA and p.group_rows == 16 and p.num_groups == 8 and p.Hkv == 8
+    assert p.head_dim == M.MHA_D and p.num_partitions == 148 // 8
+    p = M.mha_decode_plan(2, 4, 32, 4, 1000, device=-1)  # Sq * H/Hkv = 32 query rows per kv head
+    assert p.group_rows == 32
+    for args, code in (((2, 1, 12, 5, 100), 1),      # H not a multiple of Hkv
+                       ((2, 1, 8, 0, 100), 1),       # no kv heads
+                       ((2, 3, 64, 4, 100), 3),      # 3 * 16 = 48 query rows per kv head > 32
+                       ((0, 1, 8, 2, 100), 1)):
+        with pytest.raises(M.MlaError) as e:
+            M.mha_decode_plan(*args, device=-1)
+        assert e.value.code == code, args
+
+
+def test_mha_and_sink_runs_reject_without_launching(lib):
+    """Plan kinds that do not match the entry point, misaligned pointers
+    (sinks included) and short workspaces are refused on the host."""
+    mha = M.mha_decode_plan(2, 1, 8, 2, 256, device=-1)
+    mla = M.mla_decode_plan(2, 1, 16, 256, device=-1)
+    sc = ctypes.c_float(0.09)
+    run = lib.mha_decode_run
+    assert run(ctypes.byref(mla), 16, 16, 16, 16, sc, None, 16, 16, 256, mla.workspace_bytes, None) == 1
+    assert run(ctypes.byref(mha), 16, 16 + 2, 16, 16, sc, None, 16, 16, 256, mha.workspace_bytes, None) == 2
+    assert run(ctypes.byref(mha), 16, 16, 16, 16, sc, 16 + 2, 16, 16, 256, mha.workspace_bytes, None) == 2
+    assert run(ctypes.byref(mha), 16, 16, 16, 16, sc, None, 16, 16, 256, mha.workspace_bytes - 1, None) == 6
+    assert lib.mla_decode_run(ctypes.byref(mha), 16, 16, 16, sc, 16, 16, 256, mha.workspace_bytes, None) == 1
+    sinks_run = lib.mla_decode_run_sinks
+    assert sinks_run(ctypes.byref(mla), 16, 16, 16, sc, 16 + 1, 16, 16, 256, mla.workspace_bytes, None) == 2
+
+
+def test_noalloc_refuses_plans_larger_than_its_scratch(lib):
+    """A plan whose workspace exceeds the library's static scratch is refused
+    before any device call."""
+    big = M.mla_decode_plan(4096, 1, 128, 65536, device=-1, num_partitions=4096)
+    assert big.workspace_bytes > M.MLA_NOALLOC_SCRATCH_BYTES
+    rc = lib.mla_decode_run_noalloc(ctypes.byref(big), 16, 16, 16, ctypes.c_float(0.04), 16, 16, 0, None)
+    assert rc == 6
