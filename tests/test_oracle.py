@@ -82,6 +82,21 @@ def test_golden_fixture_reproduces():
     np.testing.assert_allclose(flat[idx], np.array(gold["out_value"]), rtol=0, atol=1e-12)
 
 
+def test_fp8_golden_fixture_reproduces():
+    """tests/golden/tiny_fp8_oracle.json: the FP8-cache oracle on the tiny
+    workload's quantised cache, written by tests/golden/make_golden.py."""
+    from mla_decode_attention_11_b200 import workloads as W
+    with open(os.path.join(GOLDEN, "tiny_fp8_oracle.json")) as f:
+        gold = json.load(f)
+    w = W.WORKLOADS[gold["workload"]]
+    q, codes, ks, sl = W.generate_fp8(w)
+    assert ks == gold["kv_scale"]
+    out, lse = oracle.mla_decode_fp8(q, codes, ks, sl, w.scale)
+    np.testing.assert_allclose(lse.reshape(-1), np.array(gold["lse"]), rtol=0, atol=1e-12)
+    idx = np.array(gold["out_index"], dtype=np.int64)
+    np.testing.assert_allclose(out.reshape(-1)[idx], np.array(gold["out_value"]), rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- mutants
 # CPU stand-ins of the oracle with one planted mistake each.  They are never
 # used as references; they exist only to show the pins would catch the mistake.
