@@ -83,3 +83,8 @@ def test_reference_arm_runs_on_rank_0_only(capsys, monkeypatch):
         steps, warmup, gpus = 1, 3, 2
     assert bench.run_reference(Args(), bench.W.WORKLOADS["tiny"]) is None
     assert capsys.readouterr().out == ""
+
+
+def test_l2_note_is_truthful():
+    assert bench.l2_note(604e6).startswith("inputs larger than L2")
+    assert "fits in L2" in bench.l2_note(75.5e6)
