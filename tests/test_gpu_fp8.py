@@ -24,10 +24,14 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
 
 
-def gpu_decode_fp8(q, codes, ks, sl, scale, num_partitions=0, sinks=None):
+# the FP8 kernels these tests cover (the FP8-operand kernel joins once it has run on a GPU)
+FP8_KERNELS = [M.MLA_KERNEL_FP8]
+
+
+def gpu_decode_fp8(q, codes, ks, sl, scale, num_partitions=0, sinks=None, kernel=M.MLA_KERNEL_FP8):
     plan = M.mla_decode_plan_fp8(q.shape[0], q.shape[1], q.shape[2], codes.shape[1], device=0,
-                                 num_partitions=num_partitions)
-    assert plan.kernel == M.MLA_KERNEL_FP8
+                                 num_partitions=num_partitions, kernel=kernel)
+    assert plan.kernel == kernel
     ws = M.alloc_workspace(plan)
     M.mla_decode_workspace_init(plan, ws)
     out = torch.full((q.shape[0], q.shape[1], q.shape[2], 512), float("nan"), dtype=torch.bfloat16, device=DEV)
@@ -39,9 +43,9 @@ def gpu_decode_fp8(q, codes, ks, sl, scale, num_partitions=0, sinks=None):
     return out.cpu(), lse.cpu(), plan
 
 
-def check_fp8(w, num_partitions=0, lengths=None, sinks=None, out_max_abs=OUT_MAX_ABS):
+def check_fp8(w, num_partitions=0, lengths=None, sinks=None, out_max_abs=OUT_MAX_ABS, kernel=M.MLA_KERNEL_FP8):
     q, codes, ks, sl = W.generate_fp8(w, lengths=lengths)
-    out, lse, plan = gpu_decode_fp8(q, codes, ks, sl, w.scale, num_partitions, sinks)
+    out, lse, plan = gpu_decode_fp8(q, codes, ks, sl, w.scale, num_partitions, sinks, kernel)
     ro, rl = oracle.mla_decode_fp8(q, codes, ks, sl, w.scale, sinks=sinks)
     if sinks is not None:
         # rows whose lse is a finite sink logit are not "empty" for assert_parity
@@ -58,22 +62,25 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("kernel", FP8_KERNELS)
 @pytest.mark.parametrize("name", sorted(SMALL))
-def test_fp8_small_workloads(cuda_device, name):
-    _, plan = check_fp8(SMALL[name])
+def test_fp8_small_workloads(cuda_device, name, kernel):
+    _, plan = check_fp8(SMALL[name], kernel=kernel)
     assert plan.group_rows == (16 if SMALL[name].Sq * SMALL[name].H == 16 else 32)
 
 
+@pytest.mark.parametrize("kernel", FP8_KERNELS)
 @pytest.mark.parametrize("parts", [1, 2, 37, 300])
 @pytest.mark.parametrize("H", [16, 128])
-def test_fp8_forced_partitions(cuda_device, parts, H):
-    check_fp8(W.custom(B=5, Sq=1, H=H, L=1500, L_lo=1, seed=131), num_partitions=parts)
+def test_fp8_forced_partitions(cuda_device, parts, H, kernel):
+    check_fp8(W.custom(B=5, Sq=1, H=H, L=1500, L_lo=1, seed=131), num_partitions=parts, kernel=kernel)
 
 
+@pytest.mark.parametrize("kernel", FP8_KERNELS)
 @pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 127, 128, 129, 255, 257, 1023])
-def test_fp8_lengths_around_tile_edges(cuda_device, L):
-    check_fp8(W.custom(B=2, Sq=1, H=16, L=L, seed=140 + L))
-    check_fp8(W.custom(B=1, Sq=1, H=64, L=L, seed=141 + L))
+def test_fp8_lengths_around_tile_edges(cuda_device, L, kernel):
+    check_fp8(W.custom(B=2, Sq=1, H=16, L=L, seed=140 + L), kernel=kernel)
+    check_fp8(W.custom(B=1, Sq=1, H=64, L=L, seed=141 + L), kernel=kernel)
 
 
 @pytest.mark.parametrize("H", [16, 128])
@@ -90,14 +97,15 @@ def test_fp8_head_and_token_counts(cuda_device, H, Sq):
     check_fp8(W.custom(B=2, Sq=Sq, H=H, L=600, seed=160 + H + Sq))
 
 
+@pytest.mark.parametrize("kernel", FP8_KERNELS)
 @pytest.mark.parametrize("H,parts", [(16, 0), (16, 7), (128, 0), (128, 9)])
-def test_fp8_sinks(cuda_device, H, parts):
+def test_fp8_sinks(cuda_device, H, parts, kernel):
     g = np.random.default_rng(170 + H)
     s = g.normal(0.0, 2.0, size=H).astype(np.float32)
     s[0], s[1], s[2] = -np.inf, 30.0, -50.0
     w = W.custom(B=4, Sq=1, H=H, L=900, seed=171)
     lengths = torch.tensor([900, 0, 333, 17], dtype=torch.int32)
-    check_fp8(w, num_partitions=parts, lengths=lengths, sinks=s)
+    check_fp8(w, num_partitions=parts, lengths=lengths, sinks=s, kernel=kernel)
 
 
 def test_fp8_every_finite_code(cuda_device):
