@@ -508,7 +508,7 @@ def run_fp8(args, w: W.Workload):
     torch.cuda.set_device(dev)
     q, codes, ks, sl = W.generate_fp8(w)
     qd, cd, sld = q.to(dev), codes.to(dev), sl.to(dev)
-    kernel = M.MLA_KERNEL_FP8_MMA if args.fp8_kernel == "operands" else M.MLA_KERNEL_FP8
+    kernel = M.MLA_KERNEL_FP8
     plan = M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=0, kernel=kernel)
     ws = M.alloc_workspace(plan, device=dev)
     M.mla_decode_workspace_init(plan, ws)
@@ -641,9 +641,6 @@ def main():
                     help="time the attention-sink entry point (per-head sink logits) on the same workload")
     ap.add_argument("--fp8", action="store_true",
                     help="the same MLA workload over an FP8 (E4M3) latent cache (mla_decode_run_fp8)")
-    ap.add_argument("--fp8-kernel", choices=["widen", "operands"], default="widen",
-                    help="FP8 cache kernel: codes widened to f16 (default) or the experimental "
-                         "kind::f8f6f4 operand kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -356,11 +356,14 @@ mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, 
 /*
  * mla_decode_plan_fp8_kernel -- mla_decode_plan_fp8 with an explicit kernel:
  *   kernel  0 or MLA_KERNEL_FP8: the widening kernel (what mla_decode_plan_fp8 picks);
- *           MLA_KERNEL_FP8_MMA: EXPERIMENTAL, not yet validated on a GPU -- the
- *           codes are the operands of kind::f8f6f4 MMAs and q and P are carried
- *           as sums of E4M3 terms (q: three terms of a power-of-two-scaled row,
- *           about 12 significant bits; P: two terms, about 8), so its results
- *           differ from the exact-operand path by those truncations.
+ *           MLA_KERNEL_FP8_MMA: EXPERIMENTAL -- the codes are the operands of
+ *           kind::f8f6f4 MMAs and q and P are carried as sums of E4M3 terms (q:
+ *           three terms of a power-of-two-scaled row, about 12 significant bits;
+ *           P: two terms, about 8), so its results differ from the exact-operand
+ *           path by those truncations.  Only a library built with
+ *           MLA_EXPERIMENTAL_FP8MMA defined plans it; otherwise this kernel
+ *           returns MLA_ERR_UNSUPPORTED (from the plan, and from a run given a
+ *           plan of this kind).
  *           Anything else: MLA_ERR_INVALID_ARG.
  * Other arguments and return codes as mla_decode_plan_fp8; the plan runs
  * through mla_decode_run_fp8.

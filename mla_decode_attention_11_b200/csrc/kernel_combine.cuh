@@ -34,11 +34,25 @@ struct CombineArgs {
     int split_tiles;     // 0: balanced schedule; > 0: batch-invariant chunks of this many tiles
 };
 
-// One warp per query row, 8 rows per CTA.  The kernel is bound by the bytes of
-// the partials it reads, so each lane keeps up to 4 partials x 4 float4 in
-// flight instead of walking the partials one after another.
+// Grid (B, Y): CTA (b, y) owns sequence b's query rows [y*RY, (y+1)*RY) with
+// RY = ceil(R / Y); its 8 warps take one row each at a time.  Warp 0 reads the
+// lengths once (schedule and b's unit offset in one pass), so a sequence that
+// was not cut costs its CTAs one scan and nothing else; Y is chosen by the
+// host so that about two CTAs per SM share the merging of cut sequences.
+// Within a row the kernel is bound by the bytes of the partials it reads, so
+// each lane keeps up to 4 partials x 4 float4 in flight instead of walking the
+// partials one after another.
 constexpr int kCombineThreads = 256;
-constexpr int kCombineRowsPerCta = kCombineThreads / 32;
+constexpr int kCombineWarps = kCombineThreads / 32;
+
+// CTAs per sequence along y: enough to give about two CTAs per SM when many
+// rows must be merged, never more than one per 8 rows.
+inline int combine_grid_y(int B, int R, int num_sms) {
+    const int max_y = (R + kCombineWarps - 1) / kCombineWarps;
+    int y = (2 * num_sms + B - 1) / B;
+    if (y < 1) y = 1;
+    return y < max_y ? y : max_y;
+}
 
 // DV: value width (512 for MLA, 128 for MHA); a lane owns DV / 128 float4 columns.
 template <int DV = kDv>
@@ -46,53 +60,39 @@ __global__ void __launch_bounds__(kCombineThreads)
     mla_decode_combine_kernel(const CombineArgs args) {
     static_assert(DV == 512 || DV == 128, "value width");
     constexpr int NV4 = DV / 128;  // float4 columns per lane
-    __shared__ long long red_acc[kCombineThreads / 32];
-    __shared__ long long red_tot[kCombineThreads / 32];
     __shared__ int s_split;
+    __shared__ long long s_acc, s_tot;
     const int b = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // the schedule the main kernel used for these lengths
+    // the schedule the main kernel used for these lengths, its unit count and
+    // the flat unit offset of sequence b (units: tiles, or S-tile chunks)
     if (warp == 0) {
-        const int se = schedule_scan_warp(args.seqlens, args.B, args.L_max, args.P, args.split_tiles).S;
-        if (lane == 0) s_split = se;
+        const ScheduleScan sc = schedule_scan_warp(args.seqlens, args.B, args.L_max, args.P, args.split_tiles, b);
+        if (lane == 0) {
+            s_split = sc.S;
+            s_acc = sc.acc_at;
+            s_tot = sc.units;
+        }
     }
     __syncthreads();
     const int S = s_split;
-
-    // flat unit offset of sequence b, and the total (units: tiles, or S-tile chunks)
-    long long acc = 0, tot = 0;
-    for (int i = threadIdx.x; i < args.B; i += kCombineThreads) {
-        const long long n = num_units(clamp_len(__ldg(args.seqlens + i), args.L_max, nullptr), S);
-        tot += n;
-        if (i < b) acc += n;
-    }
-    acc = warp_sum_ll(acc);
-    tot = warp_sum_ll(tot);
-    if (lane == 0) {
-        red_acc[warp] = acc;
-        red_tot[warp] = tot;
-    }
-    __syncthreads();
-    acc = 0;
-    tot = 0;
-#pragma unroll
-    for (int w = 0; w < kCombineThreads / 32; ++w) {
-        acc += red_acc[w];
-        tot += red_tot[w];
-    }
-    const int r = blockIdx.y * kCombineRowsPerCta + warp;  // this warp's query row
-    if (r >= args.R) return;
-    const size_t orow = static_cast<size_t>(b) * args.R + r;
+    const long long acc = s_acc, tot = s_tot;
+    const int rows_per = (args.R + static_cast<int>(gridDim.y) - 1) / static_cast<int>(gridDim.y);
+    const int r_lo = static_cast<int>(blockIdx.y) * rows_per;
+    const int r_hi = r_lo + rows_per < args.R ? r_lo + rows_per : args.R;
     const int L = clamp_len(__ldg(args.seqlens + b), args.L_max, nullptr);
     const long long n = num_units(L, S);
-    // a per-head sink is one more softmax term without a value (-inf: none)
-    const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
     if (n == 0) {
-        uint4* dst = reinterpret_cast<uint4*>(args.out + orow * DV);  // DV / 8 x 16 bytes
-        for (int i = lane; i < DV / 8; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
-        if (lane == 0) args.lse[orow] = sink;  // nothing to attend to: the sink alone
+        for (int r = r_lo + warp; r < r_hi; r += kCombineWarps) {
+            const size_t orow = static_cast<size_t>(b) * args.R + r;
+            // a per-head sink is one more softmax term without a value (-inf: none)
+            const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
+            uint4* dst = reinterpret_cast<uint4*>(args.out + orow * DV);  // DV / 8 x 16 bytes
+            for (int i = lane; i < DV / 8; i += 32) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+            if (lane == 0) args.lse[orow] = sink;  // nothing to attend to: the sink alone
+        }
         return;
     }
     int k, p0 = 0;
@@ -114,63 +114,67 @@ __global__ void __launch_bounds__(kCombineThreads)
         return (i == 0) ? 2 * p0 + 1 : 2 * (p0 + i);
     };
 
-    // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
-    float m = -INFINITY;
-    for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
+    for (int r = r_lo + warp; r < r_hi; r += kCombineWarps) {
+        const size_t orow = static_cast<size_t>(b) * args.R + r;
+        const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
+        // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
+        float m = -INFINITY;
+        for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    m = fmaxf(m, sink);
-    float sum = 0.f;
-    for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        m = fmaxf(m, sink);
+        float sum = 0.f;
+        for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    sum += expf(sink - m);
-    const float lse_all = m + logf(sum);
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        sum += expf(sink - m);
+        const float lse_all = m + logf(sum);
 
-    // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
-    float4 acc_o[NV4];
+        // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
+        float4 acc_o[NV4];
 #pragma unroll
-    for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i0 = 0; i0 < k; i0 += 4) {
-        float4 x[4][NV4];
-        float w[4];
+        for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = 0; i0 < k; i0 += 4) {
+            float4 x[4][NV4];
+            float w[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = i0 + j;
-            w[j] = 0.f;
-            if (i < k) {
-                const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
-                w[j] = expf(args.part_lse[prow] - lse_all);
-                const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + j;
+                w[j] = 0.f;
+                if (i < k) {
+                    const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
+                    w[j] = expf(args.part_lse[prow] - lse_all);
+                    const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
 #pragma unroll
-                for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
+                    for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
+                }
             }
-        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (i0 + j < k) {
+            for (int j = 0; j < 4; ++j) {
+                if (i0 + j < k) {
 #pragma unroll
-                for (int v = 0; v < NV4; ++v) {
-                    acc_o[v].x += w[j] * x[j][v].x;
-                    acc_o[v].y += w[j] * x[j][v].y;
-                    acc_o[v].z += w[j] * x[j][v].z;
-                    acc_o[v].w += w[j] * x[j][v].w;
+                    for (int v = 0; v < NV4; ++v) {
+                        acc_o[v].x += w[j] * x[j][v].x;
+                        acc_o[v].y += w[j] * x[j][v].y;
+                        acc_o[v].z += w[j] * x[j][v].z;
+                        acc_o[v].w += w[j] * x[j][v].w;
+                    }
                 }
             }
         }
-    }
-    __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(args.out + orow * DV);
+        __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(args.out + orow * DV);
 #pragma unroll
-    for (int v = 0; v < NV4; ++v) {
-        const int e0 = (lane + 32 * v) * 4;  // first column of acc_o[v]
-        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc_o[v].x, acc_o[v].y);
-        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc_o[v].z, acc_o[v].w);
-        uint2 pk;
-        pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-        pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-        *reinterpret_cast<uint2*>(dst + e0 / 2) = pk;
+        for (int v = 0; v < NV4; ++v) {
+            const int e0 = (lane + 32 * v) * 4;  // first column of acc_o[v]
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(acc_o[v].x, acc_o[v].y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(acc_o[v].z, acc_o[v].w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(dst + e0 / 2) = pk;
+        }
+        if (lane == 0) args.lse[orow] = lse_all;
     }
-    if (lane == 0) args.lse[orow] = lse_all;
 }
 
 }  // namespace mla

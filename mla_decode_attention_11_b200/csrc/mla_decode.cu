@@ -121,6 +121,14 @@ constexpr int kPairNV = MLA_PAIR_NV;
 constexpr int kPairNS = MLA_PAIR_NS;
 constexpr int kPairNP = MLA_PAIR_NP;  // P buffers in shared memory
 constexpr int kDefaultPrefetchTiles = 1;
+// The FP8-operand kernel (kind::f8f6f4 MMAs on the E4M3 codes) is compiled in
+// but only planned when the library is built with MLA_EXPERIMENTAL_FP8MMA,
+// until it has matched the oracle on a GPU.
+#ifdef MLA_EXPERIMENTAL_FP8MMA
+constexpr bool kFp8MmaEnabled = true;
+#else
+constexpr bool kFp8MmaEnabled = false;
+#endif
 constexpr int kDefaultSplitTiles = 16;  // batch-invariant chunks: 16 tiles = 2048 keys
 using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS, kPairNP>;
 
@@ -280,6 +288,7 @@ mla_status mla_decode_plan_fp8_kernel(int32_t B, int32_t Sq, int32_t H, int32_t 
     if (!plan) return MLA_ERR_INVALID_ARG;
     if (kernel == 0) kernel = MLA_KERNEL_FP8;
     if (kernel != MLA_KERNEL_FP8 && kernel != MLA_KERNEL_FP8_MMA) return MLA_ERR_INVALID_ARG;
+    if (kernel == MLA_KERNEL_FP8_MMA && !kFp8MmaEnabled) return MLA_ERR_UNSUPPORTED;
     mla_plan p;
     const mla_status st =
         mla_decode_plan_kernel(B, Sq, H, L_max, device, num_partitions_override, MLA_KERNEL_TRANSPOSED, &p, nullptr);
@@ -314,15 +323,17 @@ mla_status mla_decode_workspace_init(const mla_plan* plan, void* workspace, size
 
 namespace {
 
-// kv_scale: null for a bf16 cache; for an FP8 cache (plan kind MLA_KERNEL_FP8)
-// the host address of its dequantization scale
-mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
-                      float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
-                      size_t workspace_bytes, void* stream_, int phases, const float* kv_scale = nullptr) {
+// Host-side checks of a run's plan and arguments; touches no device and
+// enqueues nothing.  kv_scale: null for a bf16 cache; for an FP8 cache (plan
+// kind MLA_KERNEL_FP8) the host address of its dequantization scale.
+mla_status check_run_args(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                          float softmax_scale, const float* sinks, const void* out, const float* lse, int phases,
+                          const float* kv_scale) {
     if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
     if (!plan || !q || !kv || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
     const bool fp8 = (plan->kernel == MLA_KERNEL_FP8 || plan->kernel == MLA_KERNEL_FP8_MMA);
+    if (plan->kernel == MLA_KERNEL_FP8_MMA && !kFp8MmaEnabled) return MLA_ERR_UNSUPPORTED;
     if (fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;  // plan kind and entry point disagree
     if (fp8 && !(std::isfinite(*kv_scale) && *kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
     const mla_plan& pl = *plan;
@@ -342,9 +353,11 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16) || !aligned(lse, 4) || !aligned(seqlens, 4) ||
         !aligned(sinks, 4))
         return MLA_ERR_ALIGNMENT;
-    const Layout lay = workspace_layout(num_slots(pl), R);
-    if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+    return MLA_OK;
+}
 
+// The current device must be the plan's (when the plan names one) and an sm_100 GPU.
+mla_status check_run_device(const mla_plan& pl) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
@@ -358,6 +371,17 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
         return MLA_ERR_CUDA;
     }
     if (major != 10 || minor != 0) return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+// Encode the tensor maps and launch the requested phases; the arguments, the
+// workspace and the device have been checked.
+mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, const int32_t* seqlens,
+                         float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                         void* stream_, int phases, const float* kv_scale) {
+    const bool fp8 = (pl.kernel == MLA_KERNEL_FP8 || pl.kernel == MLA_KERNEL_FP8_MMA);
+    const int R = pl.Sq * pl.H;
+    const Layout lay = workspace_layout(num_slots(pl), R);
     EncodeTiledFn enc = encode_fn();
     if (!enc) return MLA_ERR_CUDA;
 
@@ -443,11 +467,22 @@ mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const
     c.sinks = sinks;
     c.H = pl.H;
     c.split_tiles = pl.split_tiles;
-    const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) /
-                                                                        mla::kCombineRowsPerCta));
+    const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>(mla::combine_grid_y(pl.B, R, pl.num_sms)));
     mla::mla_decode_combine_kernel<mla::kDv><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;
+}
+
+mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
+                      float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
+                      size_t workspace_bytes, void* stream, int phases, const float* kv_scale = nullptr) {
+    mla_status st = check_run_args(plan, q, kv, seqlens, softmax_scale, sinks, out, lse, phases, kv_scale);
+    if (st != MLA_OK) return st;
+    const Layout lay = workspace_layout(num_slots(*plan), plan->Sq * plan->H);
+    if (!workspace || workspace_bytes < lay.total || !aligned(workspace, 256)) return MLA_ERR_WORKSPACE;
+    st = check_run_device(*plan);
+    if (st != MLA_OK) return st;
+    return launch_phases(*plan, q, kv, seqlens, softmax_scale, sinks, out, lse, workspace, stream, phases, kv_scale);
 }
 
 }  // namespace
@@ -556,20 +591,26 @@ extern "C" {
 mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
                                   float softmax_scale, void* out, float* lse, int32_t wait_and_check,
                                   void* stream_) {
+    // every check comes before anything is enqueued, so a rejected call leaves
+    // the scratch (and an earlier call still running on it) untouched
     if (!plan) return MLA_ERR_INVALID_ARG;
     if (plan->num_partitions < 1 || plan->num_partitions > 4096 || plan->Sq < 1 || plan->H < 1)
         return MLA_ERR_INVALID_ARG;
     if (plan->split_tiles < 0 || plan->split_tiles > (1 << 17) || plan->B < 1 || plan->L_max < 1)
         return MLA_ERR_INVALID_ARG;
+    mla_status st = check_run_args(plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, 3, nullptr);
+    if (st != MLA_OK) return st;
     const size_t need = workspace_layout(num_slots(*plan), plan->Sq * plan->H).total;
     if (need > MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
+    st = check_run_device(*plan);
+    if (st != MLA_OK) return st;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) {
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }
     void* scratch = nullptr;
-    mla_status st = noalloc_scratch(dev, &scratch);
+    st = noalloc_scratch(dev, &scratch);
     if (st != MLA_OK) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     // the status words must start at zero; the partial slots are always
@@ -579,8 +620,7 @@ mla_status mla_decode_run_noalloc(const mla_plan* plan, const void* q, const voi
         cudaGetLastError();
         return MLA_ERR_CUDA;
     }
-    st = run_phases(plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, scratch, MLA_NOALLOC_SCRATCH_BYTES,
-                    stream_, 3);
+    st = launch_phases(*plan, q, kv, seqlens, softmax_scale, nullptr, out, lse, scratch, stream_, 3, nullptr);
     if (st != MLA_OK || !wait_and_check) return st;
     if (cudaStreamSynchronize(stream) != cudaSuccess) {
         cudaGetLastError();
@@ -770,8 +810,7 @@ mla_status mha_run_phases(const mla_plan* plan, const void* q, const void* k, co
     c.sinks = sinks;
     c.H = pl.H;
     c.split_tiles = pl.split_tiles;
-    const dim3 cgrid(static_cast<unsigned>(pl.B),
-                     static_cast<unsigned>((R + mla::kCombineRowsPerCta - 1) / mla::kCombineRowsPerCta));
+    const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>(mla::combine_grid_y(pl.B, R, pl.num_sms)));
     mla::mla_decode_combine_kernel<kMhaD><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
     if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
     return MLA_OK;

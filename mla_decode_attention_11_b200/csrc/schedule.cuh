@@ -87,36 +87,51 @@ __device__ __forceinline__ long long warp_sum_ll(long long v) {
 constexpr long long kCutTiles = 5;
 
 struct ScheduleScan {
-    int S;            // chunk size in tiles of this run's schedule (0: balanced over tiles)
-    long long units;  // schedule units over all sequences (tiles, or chunks)
+    int S;             // chunk size in tiles of this run's schedule (0: balanced over tiles)
+    long long units;   // schedule units over all sequences (tiles, or chunks)
+    long long acc_at;  // units of the sequences before sequence `b_at` (0 when b_at < 0)
 };
 
-// One pass over the lengths (warp-cooperative): the schedule of this run and
-// its number of units.
-__device__ inline ScheduleScan schedule_scan_warp(const int32_t* seqlens, int B, int L_max, int P, int plan_split) {
+// One pass over the lengths (warp-cooperative): the schedule of this run, its
+// number of units and, for b_at >= 0, the flat unit offset of sequence b_at.
+// Every quantity whose unit depends on the schedule is accumulated for each
+// candidate (tiles; chunks of the plan's size; non-empty sequences, the unit of
+// the one-piece-per-sequence schedule), so one pass serves all three.
+__device__ inline ScheduleScan schedule_scan_warp(const int32_t* seqlens, int B, int L_max, int P, int plan_split,
+                                                  int b_at = -1) {
     const int lane = threadIdx.x & 31;
     long long total = 0, n_max = 0, nonempty = 0, chunks = 0;
+    long long at_tiles = 0, at_nonempty = 0, at_chunks = 0;
     for (int b = lane; b < B; b += 32) {
         const int L = clamp_len(__ldg(seqlens + b), L_max, nullptr);
         const long long n = num_tiles(L);
+        const long long c = plan_split > 0 ? num_units(L, plan_split) : 0;
         total += n;
         n_max = n > n_max ? n : n_max;
         nonempty += (n > 0);
-        if (plan_split > 0) chunks += num_units(L, plan_split);
+        chunks += c;
+        if (b < b_at) {
+            at_tiles += n;
+            at_nonempty += (n > 0);
+            at_chunks += c;
+        }
     }
     total = warp_sum_ll(total);
     nonempty = warp_sum_ll(nonempty);
     chunks = warp_sum_ll(chunks);
+    at_tiles = warp_sum_ll(at_tiles);
+    at_nonempty = warp_sum_ll(at_nonempty);
+    at_chunks = warp_sum_ll(at_chunks);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         const long long y = __shfl_xor_sync(0xffffffffu, n_max, o);
         n_max = y > n_max ? y : n_max;
     }
-    if (plan_split > 0) return {plan_split, chunks};
-    if (n_max == 0 || nonempty > P || 2 * nonempty < P) return {0, total};
+    if (plan_split > 0) return {plan_split, chunks, at_chunks};
+    if (n_max == 0 || nonempty > P || 2 * nonempty < P) return {0, total, at_tiles};
     const long long T = (total + P - 1) / P;
-    if (n_max <= T + 2 * kCutTiles) return {static_cast<int>(n_max), nonempty};
-    return {0, total};
+    if (n_max <= T + 2 * kCutTiles) return {static_cast<int>(n_max), nonempty, at_nonempty};
+    return {0, total, at_tiles};
 }
 
 // Locate the first sequence overlapping flat unit `start` (warp-cooperative).

@@ -165,12 +165,23 @@ def test_fp8_run_rejects_without_launching(lib):
 
 
 def test_fp8_operand_kernel_plan_without_gpu():
-    """The experimental FP8-operand kernel is only ever chosen explicitly."""
+    """The FP8-operand kernel is not offered by the default build (it has not
+    matched the oracle on a GPU yet): an explicit request is refused as
+    unsupported, and the automatic choice is the widening kernel."""
     assert M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1).kernel == M.MLA_KERNEL_FP8
-    for H, G in ((16, 16), (128, 32)):
-        p = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8_MMA)
-        assert p.kernel == M.MLA_KERNEL_FP8_MMA and p.group_rows == G and p.cta_threads == 192
-        assert p.smem_bytes <= 232448
+    for H in (16, 128):
+        with pytest.raises(M.MlaError) as e:
+            M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8_MMA)
+        assert e.value.code == 3
+    # a hand-made plan of that kind is refused by the run entry point before
+    # anything touches a device
+    lib = M.load_library()
+    f8 = M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1)
+    f8.kernel = M.MLA_KERNEL_FP8_MMA
+    sc = ctypes.c_float(576 ** -0.5)
+    rc = lib.mla_decode_run_fp8(ctypes.byref(f8), 16, 16, ctypes.c_float(0.5), 16, sc, None, 16, 16, 256,
+                                f8.workspace_bytes, None)
+    assert rc == 3
     for bad in (1, 2, 3, 6):
         with pytest.raises(M.MlaError) as e:
             M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1, kernel=bad)
@@ -235,3 +246,25 @@ def test_noalloc_refuses_plans_larger_than_its_scratch(lib):
     assert big.workspace_bytes > M.MLA_NOALLOC_SCRATCH_BYTES
     rc = lib.mla_decode_run_noalloc(ctypes.byref(big), 16, 16, 16, ctypes.c_float(0.04), 16, 16, 0, None)
     assert rc == 6
+
+
+def test_noalloc_rejects_before_touching_the_device(lib):
+    """Every argument check of the no-allocation call comes before it touches a
+    device or enqueues the clearing of its status words, so a rejected call
+    cannot disturb an earlier call still running on the shared scratch.  On a
+    machine without a GPU the rejections therefore still name the argument
+    (a device access would have returned MLA_ERR_CUDA)."""
+    sc = ctypes.c_float(576 ** -0.5)
+    ok = M.mla_decode_plan(4, 1, 128, 1024, device=-1)
+    f8 = M.mla_decode_plan_fp8(4, 1, 16, 1024, device=-1)
+    mha = M.mha_decode_plan(4, 1, 8, 2, 1024, device=-1)
+    run = lib.mla_decode_run_noalloc
+    assert run(ctypes.byref(f8), 16, 16, 16, sc, 16, 16, 0, None) == 1     # FP8 plan on the bf16 call
+    assert run(ctypes.byref(mha), 16, 16, 16, sc, 16, 16, 0, None) == 1    # MHA plan
+    assert run(ctypes.byref(ok), 16, 16, 16, ctypes.c_float(float("nan")), 16, 16, 0, None) == 1
+    assert run(ctypes.byref(ok), 16, 16, 0, sc, 16, 16, 0, None) == 1      # no lengths
+    assert run(ctypes.byref(ok), 16 + 2, 16, 16, sc, 16, 16, 0, None) == 2  # q not 16-byte aligned
+    assert run(ctypes.byref(ok), 16, 16, 16, sc, 16 + 8, 16, 1, None) == 2  # out not 16-byte aligned
+    bad = M.mla_decode_plan(4, 1, 128, 1024, device=-1)
+    bad.group_rows = 64
+    assert run(ctypes.byref(bad), 16, 16, 16, sc, 16, 16, 0, None) == 1

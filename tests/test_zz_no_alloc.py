@@ -5,14 +5,19 @@ keeps its split-KV partials in the library's static scratch array instead of
 a caller workspace.
 
 Each case runs the call twice in a row, on different inputs, and compares
-both results with mla_decode_run (caller workspace) on the same inputs, within
-the parity tolerances of the GPU suite.  The file is collected last so it also
+both results with the fp64 oracle and with mla_decode_run (caller workspace)
+on the same inputs, within the parity tolerances of the GPU suite.  A call
+that the library rejects must enqueue nothing (checked by capturing it into a
+CUDA graph), so it cannot disturb an earlier call still running on the
+shared scratch.  The file is collected last so it also
 runs after every other GPU test has used the library in the same process; it
 passes alone in a fresh process too.
 """
 import numpy as np
 import pytest
 import torch
+
+import oracle
 
 from mla_decode_attention_11_b200 import binding as M
 from mla_decode_attention_11_b200 import workloads as W
@@ -29,6 +34,12 @@ DEV = torch.device("cuda:0")
 def _inputs(w):
     q, kv, sl = W.generate(w)
     return q.to(DEV), kv.to(DEV), sl.to(torch.int32).to(DEV)
+
+
+def _oracle(w):
+    q, kv, sl = W.generate(w)
+    ro, rl = oracle.mla_decode(q, kv, sl, w.scale)
+    return torch.from_numpy(ro), torch.from_numpy(rl)
 
 
 def _outputs(plan):
@@ -86,6 +97,8 @@ def test_noalloc_two_calls_match_workspace_run(cuda_device, name):
     M.mla_decode_run_noalloc(plan, *b, w.scale, out2, lse2, wait_and_check=True)
     _close(out1.cpu(), lse1.cpu(), *ref_a, f"{name} call 1")
     _close(out2.cpu(), lse2.cpu(), *ref_b, f"{name} call 2")
+    _close(out1.cpu(), lse1.cpu(), *_oracle(w), f"{name} call 1 vs oracle")
+    _close(out2.cpu(), lse2.cpu(), *_oracle(w2), f"{name} call 2 vs oracle")
 
     # once set up on this device, a call leaves free device memory unchanged
     out3, lse3 = _outputs(plan)
@@ -125,3 +138,41 @@ def test_noalloc_rejects_plan_beyond_scratch(cuda_device):
     assert e.value.code == 6
     torch.cuda.synchronize()
     assert torch.isnan(out.float()).all() and torch.isnan(lse).all()  # nothing was enqueued
+
+
+def test_noalloc_rejected_call_enqueues_nothing(cuda_device):
+    """A rejected call (here: an output pointer that is not 16-byte aligned,
+    and an FP8 plan on the bf16 entry point) returns its error before it
+    enqueues anything, in particular not the clearing of the shared status
+    words: captured into a CUDA graph between two torch kernels, it adds no
+    node."""
+    from cuda.bindings import runtime as rt
+    w, _ = CASES["pair_H128"]
+    plan = M.mla_decode_plan(w.B, w.Sq, w.H, w.L, device=0)
+    q, kv, sl = _inputs(w)
+    out, lse = _outputs(plan)
+    M.mla_decode_run_noalloc(plan, q, kv, sl, w.scale, out, lse, wait_and_check=True)  # device set-up
+    lib = M.load_library()
+    f8 = M.mla_decode_plan_fp8(w.B, w.Sq, 16, w.L, device=0)
+    x = torch.zeros(16, device=DEV)
+    side = torch.cuda.Stream(DEV)
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    codes = []
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            x.add_(1.0)
+            h = side.cuda_stream
+            codes.append(lib.mla_decode_run_noalloc(M.ctypes.byref(plan), q.data_ptr(), kv.data_ptr(),
+                                                    sl.data_ptr(), M.ctypes.c_float(w.scale), out.data_ptr() + 8,
+                                                    lse.data_ptr(), 0, h))
+            codes.append(lib.mla_decode_run_noalloc(M.ctypes.byref(f8), q.data_ptr(), kv.data_ptr(),
+                                                    sl.data_ptr(), M.ctypes.c_float(w.scale), out.data_ptr(),
+                                                    lse.data_ptr(), 0, h))
+            x.add_(1.0)
+    assert codes == [2, 1]
+    err, _, n = rt.cudaGraphGetNodes(g.raw_cuda_graph(), 0)
+    assert err == rt.cudaError_t.cudaSuccess
+    assert n == 2, f"the rejected calls added {n - 2} node(s) to the capture"
+    g.replay()
+    torch.cuda.synchronize()
+    assert float(x[0]) == 2.0
