@@ -67,6 +67,9 @@ def _load():
             lib.oracle_mha_decode.restype = ctypes.c_int
             lib.oracle_mha_decode.argtypes = [ptr, ptr, ptr, ptr, i64, i64, i64, i64, i64, i64, i64,
                                               dbl, ptr, ptr, ctypes.c_int]
+            lib.oracle_mha_decode_sinks.restype = ctypes.c_int
+            lib.oracle_mha_decode_sinks.argtypes = [ptr, ptr, ptr, ptr, i64, i64, i64, i64, i64, i64, i64,
+                                                    dbl, ptr, ptr, ptr, ctypes.c_int]
             lib.oracle_mla_decode_fp8_rows.restype = ctypes.c_int
             lib.oracle_mla_decode_fp8_rows.argtypes = [ptr, ptr, dbl, ptr, i64, i64, i64, i64, i64, i64,
                                                        dbl, ptr, ptr, i64, ptr, ptr, ctypes.c_int]
@@ -151,10 +154,11 @@ def mla_decode_rows(q, kv, seqlens, scale: float, row_ids, d_v: int = 512, num_t
     return out, lse
 
 
-def mha_decode(q, k, v, seqlens, scale: float, num_threads: int = 0):
+def mha_decode(q, k, v, seqlens, scale: float, num_threads: int = 0, sinks=None):
     """MHA decode oracle: q [B,Sq,H,D], k [B,L_max,Hkv,D], v [B,L_max,Hkv,Dv]
-    (bf16), seqlens int [B]; head h reads kv head h // (H // Hkv).
-    Returns (out float64 [B,Sq,H,Dv], lse float64 [B,Sq,H])."""
+    (bf16), seqlens int [B]; head h reads kv head h // (H // Hkv).  sinks None
+    or [H] per-head sink logits (one extra, value-free softmax term per head,
+    as in mla_decode).  Returns (out float64 [B,Sq,H,Dv], lse float64 [B,Sq,H])."""
     qb, kb, vb = _as_bf16_bits(q), _as_bf16_bits(k), _as_bf16_bits(v)
     if qb.ndim != 4 or kb.ndim != 4 or vb.ndim != 4:
         raise ValueError("q must be [B,Sq,H,D], k [B,L_max,Hkv,D] and v [B,L_max,Hkv,Dv]")
@@ -168,9 +172,10 @@ def mha_decode(q, k, v, seqlens, scale: float, num_threads: int = 0):
         raise ValueError("seqlens must have B entries")
     out = np.empty((B, Sq, H, Dv), dtype=np.float64)
     lse = np.empty((B, Sq, H), dtype=np.float64)
-    rc = _load().oracle_mha_decode(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, sl.ctypes.data,
-                                   B, Sq, H, Hkv, L_max, D, Dv, float(scale),
-                                   out.ctypes.data, lse.ctypes.data, int(num_threads))
+    keep, sp = _sinks_arg(sinks, H)
+    rc = _load().oracle_mha_decode_sinks(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, sl.ctypes.data,
+                                         B, Sq, H, Hkv, L_max, D, Dv, float(scale), sp,
+                                         out.ctypes.data, lse.ctypes.data, int(num_threads))
     if rc != 0:
         raise ValueError(f"oracle_mha_decode failed with code {rc}")
     return out, lse

@@ -249,17 +249,22 @@ int oracle_max_threads(void)
  *     lse[b,t,h]   = m + ln(l),   m = max_j s_j,   l = sum_j exp(s_j - m)
  *
  * Same arithmetic rules as above (exact widening, index-order sums, two
- * passes, no blocking); L = 0 gives out = 0, lse = -inf.
+ * passes, no blocking); L = 0 gives out = 0, lse = -inf.  With attention
+ * sinks the same per-head sink logit sigma_h as in the latent-cache entry
+ * point above (natural-log units, not scaled, no value) enters the max and
+ * the denominator: m = max(sigma_h, max_j s_j), l = sum_j exp(s_j - m) +
+ * exp(sigma_h - m); an empty sequence gives out = 0, lse = sigma_h.
  *   q : bf16 [B, Sq, H, D];  k : bf16 [B, L_max, Hkv, D];  v : bf16 [B, L_max, Hkv, Dv]
+ *   sinks : double [H] or NULL (no sinks)
  *   out : double [B, Sq, H, Dv];  lse : double [B, Sq, H]
  * ------------------------------------------------------------------------ */
 static void mha_one_row(const uint16_t *q_row, const uint16_t *k_seq, const uint16_t *v_seq,
-                        int64_t L, int64_t Hkv, int64_t hk, int64_t D, int64_t Dv, double scale,
+                        int64_t L, int64_t Hkv, int64_t hk, int64_t D, int64_t Dv, double scale, double sink,
                         double *scores, double *out_row, double *lse_out)
 {
     if (L <= 0) {
         for (int64_t e = 0; e < Dv; ++e) out_row[e] = 0.0;
-        *lse_out = -INFINITY;
+        *lse_out = sink;
         return;
     }
     for (int64_t j = 0; j < L; ++j) {
@@ -272,11 +277,13 @@ static void mha_one_row(const uint16_t *q_row, const uint16_t *k_seq, const uint
     double m = scores[0];
     for (int64_t j = 1; j < L; ++j)
         if (scores[j] > m) m = scores[j];
+    if (sink > m) m = sink;
     double l = 0.0;
     for (int64_t j = 0; j < L; ++j) {
         scores[j] = exp(scores[j] - m);
         l += scores[j];
     }
+    l += exp(sink - m);
     for (int64_t e = 0; e < Dv; ++e) out_row[e] = 0.0;
     for (int64_t j = 0; j < L; ++j) {
         const uint16_t *v_row = v_seq + (j * Hkv + hk) * Dv;
@@ -288,9 +295,9 @@ static void mha_one_row(const uint16_t *q_row, const uint16_t *k_seq, const uint
     *lse_out = m + log(l);
 }
 
-int oracle_mha_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *seqlens,
-                      int64_t B, int64_t Sq, int64_t H, int64_t Hkv, int64_t L_max, int64_t D, int64_t Dv,
-                      double scale, double *out, double *lse, int num_threads)
+int oracle_mha_decode_sinks(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *seqlens,
+                            int64_t B, int64_t Sq, int64_t H, int64_t Hkv, int64_t L_max, int64_t D, int64_t Dv,
+                            double scale, const double *sinks, double *out, double *lse, int num_threads)
 {
     if (!q || !k || !v || !seqlens || !out || !lse) return -1;
     if (B < 0 || Sq < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || L_max < 0 || D < 1 || Dv < 1) return -1;
@@ -315,13 +322,22 @@ int oracle_mha_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, c
             for (int64_t r = 0; r < rows; ++r) {
                 const int64_t b = r / (Sq * H);
                 const int64_t h = r % H;
+                const double sink = sinks ? sinks[h] : -INFINITY;
                 mha_one_row(q + r * D, k + b * L_max * Hkv * D, v + b * L_max * Hkv * Dv, seqlens[b], Hkv,
-                            h / group, D, Dv, scale, scores, out + r * Dv, lse + r);
+                            h / group, D, Dv, scale, sink, scores, out + r * Dv, lse + r);
             }
             free(scores);
         }
     }
     return failed ? -2 : 0;
+}
+
+int oracle_mha_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const int32_t *seqlens,
+                      int64_t B, int64_t Sq, int64_t H, int64_t Hkv, int64_t L_max, int64_t D, int64_t Dv,
+                      double scale, double *out, double *lse, int num_threads)
+{
+    return oracle_mha_decode_sinks(q, k, v, seqlens, B, Sq, H, Hkv, L_max, D, Dv, scale, NULL, out, lse,
+                                   num_threads);
 }
 
 /* ------------------------------------------------------------------------

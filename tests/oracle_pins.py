@@ -384,6 +384,82 @@ def pin_mha_single_key(impl):
 MHA_PINS = [pin_mha_mqa_equals_latent_definition, pin_mha_sdpa_library, pin_mha_head_groups, pin_mha_single_key]
 
 
+# ---------------------------------------------------------------- MHA decode with attention sinks
+# impl(q, k, v, seqlens, scale, sinks) with sinks a float64 [H] array or None.
+
+def pin_mha_sink_absent_is_minus_inf(impl):
+    """A sink of -inf changes nothing: the result equals the sink-free one,
+    bit for bit."""
+    g = torch.Generator().manual_seed(71)
+    q = _rand_bf16((2, 2, 4, 64), g)
+    k = _rand_bf16((2, 19, 2, 64), g)
+    v = _rand_bf16((2, 19, 2, 48), g)
+    sl = np.array([19, 6], np.int32)
+    o0, l0 = impl(q, k, v, sl, 0.125, None)
+    o1, l1 = impl(q, k, v, sl, 0.125, np.full(4, -np.inf))
+    np.testing.assert_array_equal(o1, o0)
+    np.testing.assert_array_equal(l1, l0)
+
+
+def pin_mha_sink_is_a_value_free_key(impl):
+    """A sink equals one more key, in the head's own kv head, whose value row
+    is zero and whose score is the sink: append key L with k = (a, 0, ..., 0)
+    and v = 0, one query head per kv head (so each kv head's extra key serves
+    exactly one head), and set sink_h = scale * q_h[0] * a exactly.  The
+    sink result over L keys must equal the sink-free result over L + 1."""
+    g = torch.Generator().manual_seed(72)
+    for L in (1, 4, 33):
+        Hkv = 3
+        q = _rand_bf16((1, 1, Hkv, 32), g)
+        k = _rand_bf16((1, L + 1, Hkv, 32), g)
+        v = _rand_bf16((1, L + 1, Hkv, 16), g)
+        k[0, L] = 0
+        v[0, L] = 0
+        a = torch.tensor([1.5, -2.0, 3.25], dtype=torch.bfloat16)
+        k[0, L, :, 0] = a
+        scale = 0.25
+        sinks = np.array([scale * float(q[0, 0, h, 0]) * float(a[h]) for h in range(Hkv)])
+        o_s, l_s = impl(q, k, v, np.array([L], np.int32), scale, sinks)
+        o_k, l_k = impl(q, k, v, np.array([L + 1], np.int32), scale, None)
+        np.testing.assert_allclose(o_s, o_k, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(l_s, l_k, rtol=0, atol=1e-12)
+
+
+def pin_mha_sink_zero_query(impl):
+    """q = 0: all scores are 0, so the weights are 1 / (L + e^sigma): out =
+    mean of the kv head's values * L / (L + e^sigma), lse = ln(L + e^sigma),
+    with a sink far above the scores (e^800 overflows a double, so the sink
+    must take part in the max)."""
+    g = torch.Generator().manual_seed(73)
+    H, Hkv, L = 4, 2, 11
+    q = torch.zeros((1, 1, H, 32), dtype=torch.bfloat16)
+    k = _rand_bf16((1, L, Hkv, 32), g)
+    v = _rand_bf16((1, L, Hkv, 24), g)
+    sinks = np.array([-2.0, 0.5, 3.0, 800.0])
+    out, lse = impl(q, k, v, np.array([L], np.int32), 0.3, sinks)
+    for h, sg in enumerate(sinks):
+        mean = v[0, :, h // 2].double().mean(dim=0).numpy()
+        ref_lse = max(sg, math.log(L)) + math.log1p(math.exp(-abs(sg - math.log(L))))
+        np.testing.assert_allclose(out[0, 0, h], mean * math.exp(math.log(L) - ref_lse), rtol=1e-12, atol=1e-300)
+        assert abs(lse[0, 0, h] - ref_lse) <= 1e-12 * max(1.0, abs(ref_lse))
+
+
+def pin_mha_sink_empty_sequence(impl):
+    """L = 0: out = 0 and the log-sum-exp is the head's sink alone."""
+    g = torch.Generator().manual_seed(74)
+    q = _rand_bf16((2, 1, 2, 32), g)
+    k = _rand_bf16((2, 5, 1, 32), g)
+    v = _rand_bf16((2, 5, 1, 32), g)
+    sinks = np.array([0.75, -4.0])
+    out, lse = impl(q, k, v, np.array([0, 5], np.int32), 0.2, sinks)
+    np.testing.assert_array_equal(out[0], 0.0)
+    np.testing.assert_array_equal(lse[0, 0], sinks)
+
+
+MHA_SINK_PINS = [pin_mha_sink_absent_is_minus_inf, pin_mha_sink_is_a_value_free_key, pin_mha_sink_zero_query,
+                 pin_mha_sink_empty_sequence]
+
+
 # ---------------------------------------------------------------- FP8 latent cache
 # FP8 pins take (decode, attend): decode(codes uint8 array) -> float64 values
 # of the E4M3 codes; attend(q, codes, kv_scale, seqlens, scale, d_v, sinks)

@@ -270,6 +270,70 @@ def test_mha_pins_catch_planted_mistakes(name):
         assert failed, f"planted mistake '{name}' passed every MHA pin"
 
 
+# ---------------------------------------------------------------- MHA decode oracle with sinks
+
+@pytest.mark.parametrize("pin", pins.MHA_SINK_PINS, ids=lambda p: p.__name__)
+def test_mha_oracle_sink_pin(pin):
+    pin(lambda q, k, v, sl, scale, sinks: oracle.mha_decode(q, k, v, sl, scale, sinks=sinks))
+
+
+def _np_mha_sinks(q, k, v, sl, scale, sinks, *, sink_mode="correct"):
+    qd, kd, vd = (x.to(torch.float64).numpy() for x in (q, k, v))
+    B, Sq, H, D = qd.shape
+    Hkv, Dv = kd.shape[2], vd.shape[3]
+    out = np.zeros((B, Sq, H, Dv))
+    lse = np.zeros((B, Sq, H))
+    for b in range(B):
+        L = int(sl[b])
+        for t in range(Sq):
+            for h in range(H):
+                hk = h // (H // Hkv)
+                sg = -np.inf if sinks is None else float(sinks[0 if sink_mode == "first_head" else h])
+                if sink_mode == "scaled":
+                    sg *= scale
+                if L == 0:
+                    lse[b, t, h] = -np.inf if sink_mode == "empty_minus_inf" else sg
+                    continue
+                s = (kd[b, :L, hk] @ qd[b, t, h]) * scale
+                m = s.max() if sink_mode == "not_in_max" else max(s.max(), sg)
+                w = np.exp(s - m)
+                l = w.sum() + (0.0 if sink_mode == "ignored" else np.exp(sg - m))
+                o = w @ vd[b, :L, hk]
+                if sink_mode == "carries_first_value":
+                    o = o + np.exp(sg - m) * vd[b, 0, hk]
+                out[b, t, h] = o / l
+                lse[b, t, h] = m + np.log(l)
+    return out, lse
+
+
+MHA_SINK_MUTANTS = {
+    "correct": {},
+    "sink_ignored": dict(sink_mode="ignored"),
+    "sink_multiplied_by_scale": dict(sink_mode="scaled"),
+    "sink_left_out_of_max": dict(sink_mode="not_in_max"),
+    "sink_carries_a_value": dict(sink_mode="carries_first_value"),
+    "first_head_sink_for_all": dict(sink_mode="first_head"),
+    "empty_sequence_lse_minus_inf": dict(sink_mode="empty_minus_inf"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MHA_SINK_MUTANTS))
+def test_mha_sink_pins_catch_planted_mistakes(name):
+    def impl(q, k, v, sl, scale, sinks):
+        return _np_mha_sinks(q, k, v, sl, scale, sinks, **MHA_SINK_MUTANTS[name])
+    failed = []
+    for pin in pins.MHA_SINK_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(impl)
+        except AssertionError:
+            failed.append(pin.__name__)
+    if name == "correct":
+        assert failed == [], f"a correct stand-in must pass every MHA sink pin, failed: {failed}"
+    else:
+        assert failed, f"planted mistake '{name}' passed every MHA sink pin"
+
+
 # ---------------------------------------------------------------- FP8 latent cache oracle
 
 def _oracle_fp8_attend(q, codes, ks, sl, scale, d_v, sinks):
