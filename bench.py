@@ -53,7 +53,9 @@ def whole_job_rate(world: int, units_per_rank: float, ms: float) -> float:
     return world * units_per_rank / (ms * 1e-3)
 
 
-L2_BYTES = 126e6  # B200 L2
+L2_BYTES = 126e6  # B200 L2 (the device's own size is read at run time where it matters)
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}  # HBM3e and dense bf16, nominal
+MAX_PLAUSIBLE_FRAC = 1.2  # a roofline fraction above this means the timed kernel skipped work
 
 
 def l2_note(cache_bytes: float) -> str:
@@ -62,6 +64,41 @@ def l2_note(cache_bytes: float) -> str:
     if cache_bytes > L2_BYTES:
         return "inputs larger than L2 (kv %.0f MB > 126 MB), no flush" % (cache_bytes / 1e6)
     return "kv %.0f MB fits in L2 (126 MB), no flush: steps after the first may hit L2" % (cache_bytes / 1e6)
+
+
+def needs_flush(cache_bytes: float, l2_bytes: float) -> bool:
+    """Flush L2 between timed decodes unless the cache streamed per decode is
+    at least twice the L2 size (then a decode evicts its own inputs)."""
+    return cache_bytes < 2 * l2_bytes
+
+
+def flush_note(cache_bytes: float, l2_bytes: float) -> str:
+    return ("kv %.0f MB < 2 x L2 (%.0f MB): L2 flushed (a %.0f MB write) before every timed decode, each decode "
+            "timed by its own events" % (cache_bytes / 1e6, l2_bytes / 1e6, 2 * l2_bytes / 1e6))
+
+
+def compare_rows(out_rows, lse_rows, ref_out, ref_lse) -> dict:
+    """Parity of the timed run's own outputs against the oracle on the rows the
+    CPU baseline computed (the tolerances of the parity tests)."""
+    import numpy as np
+    o = np.asarray(out_rows, dtype=np.float64).reshape(ref_out.shape)
+    d = o - ref_out
+    max_abs = float(np.abs(d).max()) if d.size else 0.0
+    rel = float(np.linalg.norm(d) / max(np.linalg.norm(ref_out), 1e-300))
+    lg = np.asarray(lse_rows, dtype=np.float64).reshape(-1)
+    lr = ref_lse.reshape(-1)
+    fin = np.isfinite(lr)
+    lse_err = float(np.abs(lg[fin] - lr[fin]).max()) if fin.any() else 0.0
+    ok = bool(np.all(np.isfinite(o)) and max_abs <= 2e-2 and rel <= 5e-3 and lse_err <= 1e-3
+              and np.array_equal(np.isfinite(lg), fin))
+    return {"rows": int(ref_out.shape[0]), "max_abs": max_abs, "rel_l2": rel, "lse_max_abs": lse_err,
+            "tolerance": "max-abs 2e-2, rel-L2 5e-3, lse 1e-3", "ok": ok}
+
+
+def refuse(line: dict, why: str) -> None:
+    """A number that cannot be right is not printed as a result."""
+    sys.stderr.write("bench.py: refusing to report this measurement: %s\n%s\n" % (why, json.dumps(line)))
+    sys.exit(1)
 
 
 def load_peaks():
@@ -145,7 +182,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.0005)
 
     def start(self):
         if self.ok:
@@ -162,17 +199,21 @@ class ClockSampler:
                 "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
 
 
-def cpu_oracle_sample(w: W.Workload, q, kv, sl, seqs):
-    """Time the oracle, as it stands, on whole sequences `seqs` (all heads)."""
+def cpu_oracle_sample(w: W.Workload, q, kv, sl, seqs, num_threads: int = 0, keep: bool = False):
+    """Time the oracle, as it stands, on whole sequences `seqs` (all heads);
+    with keep, also return its rows (out [n, 512], lse [n]) and their ids."""
     import numpy as np
     import oracle
     R = w.Sq * w.H
     rows = np.concatenate([np.arange(b * R, (b + 1) * R) for b in seqs]).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.mla_decode_rows(q, kv, sl, w.scale, rows)
+    ro, rl = oracle.mla_decode_rows(q, kv, sl, w.scale, rows, num_threads=num_threads)
     dt = time.perf_counter() - t0
     flops = sum(int(sl[b]) for b in seqs) * R * 2 * (W.D_QK + W.D_V)
-    return flops, dt, oracle.max_threads()
+    threads = num_threads if num_threads > 0 else oracle.max_threads()
+    if keep:
+        return flops, dt, threads, (rows, ro, rl)
+    return flops, dt, threads
 
 
 def run_reference(args, w: W.Workload):
@@ -246,9 +287,18 @@ def run_ours(args, w: W.Workload):
             step()
     M.mla_decode_check(plan, ws, stream=stream)
 
-    # The K timed decodes are launched as one CUDA graph (captured, not run,
-    # here), so that the host-side cost of a call (~25 us through Python)
-    # does not leave the GPU idle between the launches of small workloads.
+    # Inputs larger than twice L2 are streamed as they are; a smaller cache gets
+    # an L2 flush (a write of twice the L2 size) before every timed decode, and
+    # each decode is then timed by its own pair of events.
+    l2_bytes = float(torch.cuda.get_device_properties(dev).L2_cache_size)
+    cache_bytes = kv.numel() * 2
+    flush_buf = torch.empty(int(2 * l2_bytes), dtype=torch.uint8, device=dev) \
+        if needs_flush(cache_bytes, l2_bytes) else None
+
+    # Without a flush the K timed decodes are launched as one CUDA graph
+    # (captured, not run, here), so that the host-side cost of a call (~25 us
+    # through Python) does not leave the GPU idle between the launches of small
+    # workloads.
     def capture(fn, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
@@ -257,7 +307,21 @@ def run_ours(args, w: W.Workload):
                     fn()
         return g
 
-    g_steps = capture(step, args.steps)
+    def flushed_ms(fn, n):
+        """Mean device time of fn over n calls, L2 flushed before each; a GPU
+        sleep in front lets the host enqueue all of it before it starts."""
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(int(20e6 + 2e6 * n))
+            for i in range(n):
+                flush_buf.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                fn()
+                evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in evs) / n
+
+    g_steps = capture(step, args.steps) if flush_buf is None else None
     torch.cuda.synchronize(dev)
 
     # ---- timed region: K full steps
@@ -266,27 +330,34 @@ def run_ours(args, w: W.Workload):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):  # a graph replays on the current stream
-        e0.record(stream)
-        g_steps.replay()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
+    if flush_buf is None:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):  # a graph replays on the current stream
+            e0.record(stream)
+            g_steps.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        t_ms = e0.elapsed_time(e1) / args.steps
+    else:
+        t_ms = flushed_ms(step, args.steps)
     clk = clocks.stop()
     if dist:
         dist.barrier()
-    t_ms = e0.elapsed_time(e1) / args.steps
     M.mla_decode_check(plan, ws, stream=stream)
+    out_timed, lse_timed = out.cpu(), lse.cpu()  # the timed run's own result, checked below
     t_ms = max_over_ranks(t_ms, dist, dev)
 
-    # ---- per-kernel breakdown: the same launches, each kernel alone, back to
-    # back in a graph (phase 1 = main kernel, phase 2 = split-KV combine)
+    # ---- per-kernel breakdown: the same launches, each kernel alone (phase 1 =
+    # main kernel, phase 2 = split-KV combine), back to back in a graph, or one
+    # by one after a flush as above
     n_brk = max(3, min(args.steps, 50))
 
-    def timed_graph(phase):
-        g = capture(lambda: M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, phase, stream=stream),
-                    n_brk)
+    def phase_ms(phase):
+        fn = lambda: M.mla_decode_run_phase(plan, qd, kvd, sld, w.scale, out, lse, ws, phase, stream=stream)
+        if flush_buf is not None:
+            return flushed_ms(fn, n_brk)
+        g = capture(fn, n_brk)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             a.record(stream)
@@ -295,8 +366,8 @@ def run_ours(args, w: W.Workload):
         torch.cuda.synchronize(dev)
         return a.elapsed_time(b) / n_brk
 
-    main_avg = timed_graph(1)
-    comb_avg = timed_graph(2)
+    main_avg = phase_ms(1)
+    comb_avg = phase_ms(2)
     del g_steps
     M.mla_decode_check(plan, ws, stream=stream)
 
@@ -335,23 +406,40 @@ def run_ours(args, w: W.Workload):
     if bound == "hbm":
         achieved = nbytes / (main_avg * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
+        spec = SPEC_PEAKS["hbm_gbs"]
         unit = "GB/s"
     else:
         achieved = flops / (main_avg * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
+        spec = SPEC_PEAKS["bf16_tflops"]
         unit = "TFLOP/s"
     roof_time_ms = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e3
     # the record was taken with the default plan; a batch-invariant plan moves other bytes
     traffic, traffic_note = load_traffic(w.name) if not plan.split_tiles else (None, None)
 
     cpu_base = None
+    check = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        # the whole workload once (~4 s on 16 host cores for the headline line)
-        seqs = list(range(w.B))
-        f_cpu, dt_cpu, cores = cpu_oracle_sample(w, q, kv, sl, seqs)
+        # the oracle on the whole workload once (~4 s on 16 host cores for the
+        # headline line, or a bounded number of sequences of larger ones); its
+        # rows double as the check of the timed run's own outputs
+        R = w.Sq * w.H
+        per_seq = float(sl.to(torch.float64).mean()) * R * 2 * (W.D_QK + W.D_V)
+        n_seq = max(1, min(w.B, int(4e11 / per_seq)))  # 0.4 TFLOP of fp64 work at most (~10 s)
+        seqs = list(range(n_seq))
+        f_cpu, dt_cpu, cores, (rows, ro, rl) = cpu_oracle_sample(w, q, kv, sl, seqs, keep=True)
         cpu_base = {"value": f_cpu / dt_cpu / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                    "sample": f"{len(seqs)} of {w.B} sequences, all {w.Sq * w.H} query rows, "
+                    "sample": f"{len(seqs)} of {w.B} sequences, all {R} query rows, "
                               f"{dt_cpu:.1f} s of fp64 CPU work"}
+        if w.name in ("tiny", "dsv3"):
+            # per-core context: the same oracle on one host thread, one sequence
+            f1, dt1, _ = cpu_oracle_sample(w, q, kv, sl, [0], num_threads=1)
+            cpu_base["single_core"] = {"value": f1 / dt1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                                       "sample": f"1 sequence, all {R} query rows, {dt1:.2f} s"}
+        check = compare_rows(out_timed.reshape(-1, W.D_V)[rows].to(torch.float64).numpy(),
+                             lse_timed.reshape(-1)[rows].to(torch.float64).numpy(), ro, rl)
+        if args.sinks:  # the oracle rows above have no sinks; the sink path is checked by the tests
+            check = {"skipped": "sink decode: the CPU-baseline rows have no sinks"}
 
     if rank == 0:
         line = {
@@ -364,11 +452,12 @@ def run_ours(args, w: W.Workload):
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "kernel": {1: "transposed", 2: "pair"}.get(plan.kernel, str(plan.kernel)),
                        "group_rows": plan.group_rows, "partitions": plan.num_partitions,
-                       "l2": l2_note(kv.numel() * 2)},
+                       "l2": flush_note(cache_bytes, l2_bytes) if flush_buf is not None else l2_note(cache_bytes)},
             "hbm_gbs": hbm_gbs,
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else peak_src,
+                         "spec_peak": spec, "frac_of_spec": achieved / spec,
                          "kernel": "mla_decode_transposed_kernel" if plan.kernel == 1 else "mla_decode_pair_kernel",
                          "kernel_ms": main_avg, "combine_ms": comb_avg,
                          "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
@@ -380,11 +469,18 @@ def run_ours(args, w: W.Workload):
             "gpu_launches": 2 * args.steps,
             "clocks": clk,
             "cpu_baseline": cpu_base,
+            "output_check": check,
         }
-        print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
+    if rank == 0:
+        frac = achieved / peak
+        if not (0.0 < frac <= MAX_PLAUSIBLE_FRAC):
+            refuse(line, f"roofline fraction {frac:.3f} is outside (0, {MAX_PLAUSIBLE_FRAC}]")
+        if check is not None and check.get("ok") is False:
+            refuse(line, "the timed run's outputs do not match the oracle")
+        print(json.dumps(line), flush=True)
 
 
 def run_mha(args, w: W.MhaWorkload):

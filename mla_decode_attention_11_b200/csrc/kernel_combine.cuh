@@ -117,47 +117,92 @@ __global__ void __launch_bounds__(kCombineThreads)
     for (int r = r_lo + warp; r < r_hi; r += kCombineWarps) {
         const size_t orow = static_cast<size_t>(b) * args.R + r;
         const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
-        // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
-        float m = -INFINITY;
-        for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        m = fmaxf(m, sink);
-        float sum = 0.f;
-        for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        sum += expf(sink - m);
-        const float lse_all = m + logf(sum);
-
-        // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
         float4 acc_o[NV4];
-#pragma unroll
-        for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i0 = 0; i0 < k; i0 += 4) {
+        float lse_all;
+        if (k <= 4) {
+            // up to 4 pieces: every lane loads all their lse values and its
+            // columns of all their partial rows at once (one round trip)
+            float pl[4];
             float4 x[4][NV4];
-            float w[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int i = i0 + j;
-                w[j] = 0.f;
-                if (i < k) {
-                    const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
-                    w[j] = expf(args.part_lse[prow] - lse_all);
+                pl[j] = -INFINITY;
+                if (j < k) {
+                    const size_t prow = static_cast<size_t>(slot_of(j)) * args.R + r;
+                    pl[j] = args.part_lse[prow];
                     const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
 #pragma unroll
                     for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
                 }
             }
+            float m = sink;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) m = fmaxf(m, pl[j]);
+            float w[4], sum = expf(sink - m);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                if (i0 + j < k) {
+                w[j] = (j < k) ? expf(pl[j] - m) : 0.f;
+                sum += w[j];
+            }
+            lse_all = m + logf(sum);
+            const float inv = 1.f / sum;
+#pragma unroll
+            for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < k) {
+                    const float wj = w[j] * inv;
 #pragma unroll
                     for (int v = 0; v < NV4; ++v) {
-                        acc_o[v].x += w[j] * x[j][v].x;
-                        acc_o[v].y += w[j] * x[j][v].y;
-                        acc_o[v].z += w[j] * x[j][v].z;
-                        acc_o[v].w += w[j] * x[j][v].w;
+                        acc_o[v].x += wj * x[j][v].x;
+                        acc_o[v].y += wj * x[j][v].y;
+                        acc_o[v].z += wj * x[j][v].z;
+                        acc_o[v].w += wj * x[j][v].w;
+                    }
+                }
+            }
+        } else {
+            // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
+            float m = -INFINITY;
+            for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            m = fmaxf(m, sink);
+            float sum = 0.f;
+            for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            sum += expf(sink - m);
+            lse_all = m + logf(sum);
+
+            // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
+#pragma unroll
+            for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int i0 = 0; i0 < k; i0 += 4) {
+                float4 x[4][NV4];
+                float w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = i0 + j;
+                    w[j] = 0.f;
+                    if (i < k) {
+                        const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
+                        w[j] = expf(args.part_lse[prow] - lse_all);
+                        const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
+#pragma unroll
+                        for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (i0 + j < k) {
+#pragma unroll
+                        for (int v = 0; v < NV4; ++v) {
+                            acc_o[v].x += w[j] * x[j][v].x;
+                            acc_o[v].y += w[j] * x[j][v].y;
+                            acc_o[v].z += w[j] * x[j][v].z;
+                            acc_o[v].w += w[j] * x[j][v].w;
+                        }
                     }
                 }
             }

@@ -89,7 +89,8 @@ struct PairCfg {
 template <int NK, int NV, int NS, int NP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v, const MainArgs args) {
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                           const __grid_constant__ CUtensorMap tm_part, const MainArgs args) {
     using C = PairCfg<NK, NV, NS, NP>;
     extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -180,6 +181,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
+        ptx::prefetch_tmap(&tm_out);
+        ptx::prefetch_tmap(&tm_part);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -279,6 +282,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 ++piece_cnt;
             }
             if (!ok) atomicOr(args.status, kStatusTimeout);
+            // before teardown, every load this CTA pair may still have in flight
+            // must have landed: the leader counts both CTAs' bytes, so it waits
+            // (bounded) for the last phase it armed on each K slot and on Q
+            if (leader) {
+                const uint32_t n_k = k_cnt < static_cast<uint32_t>(NK) ? k_cnt : static_cast<uint32_t>(NK);
+                for (uint32_t i = 0; i < n_k; ++i) {
+                    const uint32_t c = k_cnt - 1 - i;
+                    ptx::mbar_wait_bounded(k_full + c % NK, (c / NK) & 1, tmo);
+                }
+                if (piece_cnt > 0) ptx::mbar_wait_bounded(q_full, (piece_cnt - 1) & 1, tmo);
+            }
         }
         __syncwarp();
     } else if (warp == 5) {
@@ -306,6 +320,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 }
             }
             if (!ok) atomicOr(args.status, kStatusTimeout);
+            if (leader) {  // as for K: the last armed phase of each V slot has landed
+                const uint32_t n_v = v_cnt < static_cast<uint32_t>(NV) ? v_cnt : static_cast<uint32_t>(NV);
+                for (uint32_t i = 0; i < n_v; ++i) {
+                    const uint32_t c = v_cnt - 1 - i;
+                    ptx::mbar_wait_bounded(v_full + c % NV, (c / NV) & 1, tmo);
+                }
+            }
         }
         __syncwarp();
     } else if (warp == 6) {
@@ -432,6 +453,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
         uint32_t tile_cnt = 0, sync_cnt = 0;
         bool ok = true;
+        // scores are scaled by cs before exp2; a non-positive scale is applied to
+        // the raw scores up front (cs = 1 after that), so that the row max of the
+        // raw scores times cs is the scaled row max
+        const float scale_log2 = args.scale_log2;
         auto group_barrier = [&]() -> bool {
             ptx::mbar_arrive(group_sync);
             const bool rr = ptx::mbar_wait_bounded(group_sync, sync_cnt & 1, tmo);
@@ -440,8 +465,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         };
         Piece pc;
         while (ok && walker.next(pc)) {
-            float m_ref = -INFINITY;
-            float l_part = 0.f;
+            float m_ref = -INFINITY;  // reference max (base 2) of the row, the same in both of its threads
+            float l_part = 0.f;       // this thread's share of the row sum, relative to m_ref
             for (int t = pc.tile_lo; t < pc.tile_hi; ++t) {
                 const bool first = (t == pc.tile_lo);
                 int row0 = t * kTileKV;
@@ -460,43 +485,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int kv = kv0 + j;
-                        x[j] = (kv >= lo && kv < pc.L) ? __uint_as_float(ra[j]) * args.scale_log2 : -INFINITY;
-                        const int kv2 = kv0 + 32 + j;
-                        x[32 + j] = (kv2 >= lo && kv2 < pc.L) ? __uint_as_float(rb[j]) * args.scale_log2 : -INFINITY;
+                        x[j] = __uint_as_float(ra[j]);
+                        x[32 + j] = __uint_as_float(rb[j]);
                     }
                 }
-                float mloc = x[0];
+                float cs = scale_log2;
+                if (!(cs > 0.f)) {
 #pragma unroll
-                for (int j = 1; j < 64; ++j) mloc = fmaxf(mloc, x[j]);
+                    for (int j = 0; j < 64; ++j) x[j] *= cs;
+                    cs = 1.f;
+                }
+                // only the end-aligned last tile of a sequence holds keys of the
+                // previous tile (below lo); every key of a tile is below L
+                if (row0 < lo) {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (kv0 + j < lo) x[j] = -INFINITY;
+                }
+                // this thread's max (pairwise tree), then published for the row's
+                // other thread; the exchange completes while the exps below run
+                float mt[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mt[j] = fmaxf(x[2 * j], x[2 * j + 1]);
+#pragma unroll
+                for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
+                const float mloc = mt[0] * cs;
                 float* redmax = red + (tile_cnt & 1) * 128;
                 redmax[L_id] = mloc;
-                ok = group_barrier();
+                ptx::mbar_arrive(group_sync);
+                // P[r][64h .. 64h+63] = exp2(x * cs - m_ref) as bf16.  Past a
+                // piece's first tile the reference max is known before this
+                // tile's max, so P is computed at once; it is redone only when
+                // the row max outgrew the reference by more than 8 (p <= 2^8).
+                uint32_t packed[32];
+                float lsum = 0.f;
+                auto exps = [&](float m) {
+                    lsum = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float a0 = ex2_approx(fmaf(x[2 * e], cs, -m));
+                        const float a1 = ex2_approx(fmaf(x[2 * e + 1], cs, -m));
+                        lsum += a0 + a1;
+                        const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
+                        packed[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                    }
+                };
+                if (!first) exps(m_ref);
+                ok = ptx::mbar_wait_bounded(group_sync, sync_cnt & 1, tmo);
+                ++sync_cnt;
                 if (!ok) break;
                 const float mrow = fmaxf(mloc, redmax[L_id ^ 64]);
-                // reference max: the tile's row max on a piece's first tile, else
-                // raised lazily only when the row max grew by more than 8 (p <= 2^8)
                 float alpha = 1.f;
                 bool grow = false;
                 if (first) {
                     m_ref = mrow;
+                    exps(m_ref);
                 } else if (mrow > m_ref + 8.f) {
                     grow = true;
                     alpha = ex2_approx(m_ref - mrow);
                     m_ref = mrow;
                     l_part *= alpha;
+                    exps(m_ref);
                 }
+                l_part += lsum;
                 const bool warp_grow = __any_sync(0xffffffffu, grow);
-                // P[r][64h .. 64h+63] = exp2(x - m_ref) as bf16, computed before waiting
-                uint32_t packed[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const float a0 = ex2_approx(x[2 * e] - m_ref);
-                    const float a1 = ex2_approx(x[2 * e + 1] - m_ref);
-                    l_part += a0 + a1;
-                    const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
-                    packed[e] = *reinterpret_cast<const uint32_t*>(&hv);
-                }
                 const uint32_t pb = (NP == 2) ? (tile_cnt & 1) : 0;
                 // the P buffer is free once the PV that last read it completed
                 // (NP = 1: the previous tile's; NP = 2: the one two tiles back)
@@ -558,64 +612,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             if (args.sinks != nullptr && pc.slot < 0)
                 o_fac = fold_sink(m_ref, l_row, args.sinks[qrow % args.H] * kLog2e);
             const float inv_l = o_fac / l_row;
-            // O / l leaves TMEM 64 columns at a time and is transposed through a
-            // warp-private 32 x 64 fp32 stage, so that each store instruction
-            // writes whole row segments (a thread holds one row, and direct
-            // stores would put 32 rows in every instruction).  The stage is the
-            // P buffers: every PV of the piece has completed, and the next
-            // piece's P is written only after the closing group barrier.
-            {
-                float4* stage = reinterpret_cast<float4*>(p_smem) + warp * (32 * 16);
-                const int row_base = g * 128 + static_cast<int>(rank) * 64 + 32 * (warp & 1);  // lane 0's row
-                const bool partial = (pc.slot >= 0);
-                const size_t grow0 =
-                    partial ? static_cast<size_t>(pc.slot) * args.R + row_base : static_cast<size_t>(pc.b) * args.R + row_base;
-#pragma unroll 1
-                for (int blk = 0; blk < 4; ++blk) {
-                    const int i = blk >> 1, c0 = (blk & 1) * 64;
-                    uint32_t ra[32], rb[32];
-                    ptx::tmem_ld_32(lane_addr + 128 * i + c0, ra);
-                    ptx::tmem_ld_32(lane_addr + 128 * i + c0 + 32, rb);
-                    ptx::tmem_wait_ld();
-                    float4* srow = stage + lane * 16;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        srow[k ^ (lane & 15)] =
-                            make_float4(__uint_as_float(ra[4 * k + 0]) * inv_l, __uint_as_float(ra[4 * k + 1]) * inv_l,
-                                        __uint_as_float(ra[4 * k + 2]) * inv_l, __uint_as_float(ra[4 * k + 3]) * inv_l);
-                        srow[(k + 8) ^ (lane & 15)] =
-                            make_float4(__uint_as_float(rb[4 * k + 0]) * inv_l, __uint_as_float(rb[4 * k + 1]) * inv_l,
-                                        __uint_as_float(rb[4 * k + 2]) * inv_l, __uint_as_float(rb[4 * k + 3]) * inv_l);
-                    }
-                    __syncwarp();
-                    const int col = 256 * i + 128 * h + c0;  // first value column of the block
-                    if (partial) {
-                        // 16 lanes per row: 2 rows x 256 B per instruction
-#pragma unroll
-                        for (int it = 0; it < 16; ++it) {
-                            const int rr = 2 * it + (lane >> 4), k = lane & 15;
-                            const float4 x = stage[rr * 16 + (k ^ (rr & 15))];
-                            *reinterpret_cast<float4*>(args.part_o + (grow0 + rr) * kDv + col + 4 * k) = x;
-                        }
-                    } else {
-                        // 8 lanes per row, 8 columns each: 4 rows x 128 B of bf16 per instruction
-#pragma unroll
-                        for (int it = 0; it < 8; ++it) {
-                            const int rr = 4 * it + (lane >> 3), k = lane & 7;
-                            const float4 x0 = stage[rr * 16 + ((2 * k) ^ (rr & 15))];
-                            const float4 x1 = stage[rr * 16 + ((2 * k + 1) ^ (rr & 15))];
-                            const __nv_bfloat162 b0 = __floats2bfloat162_rn(x0.x, x0.y);
-                            const __nv_bfloat162 b1 = __floats2bfloat162_rn(x0.z, x0.w);
-                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x1.x, x1.y);
-                            const __nv_bfloat162 b3 = __floats2bfloat162_rn(x1.z, x1.w);
-                            *reinterpret_cast<uint4*>(args.out + (grow0 + rr) * kDv + col + 8 * k) =
-                                make_uint4(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1),
-                                           *reinterpret_cast<const uint32_t*>(&b2), *reinterpret_cast<const uint32_t*>(&b3));
-                        }
-                    }
-                    __syncwarp();  // the stage is rewritten by the next block
-                }
-            }
             if (h == 0) {
                 const float lse_nat = (m_ref + log2f(l_row)) * 0.69314718055994530942f;
                 if (pc.slot < 0)
@@ -623,10 +619,70 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 else
                     args.part_lse[static_cast<size_t>(pc.slot) * args.R + qrow] = lse_nat;
             }
+            // O / l leaves TMEM one 128-byte column block at a time: this warp's
+            // 32 rows x 128 bytes are written into a 4 KB stage in the 128-byte
+            // swizzle a TMA store expects (lane = row, so each instruction
+            // spreads over all banks), and one lane stores the box with TMA.
+            // Each warp owns 8 KB of the P buffers (two stages, alternating):
+            // every PV of the piece has completed, and the next piece's P is
+            // written only after the closing group barrier.
+            {
+                uint8_t* stage = p_smem + warp * 8192;
+                const bool partial = (pc.slot >= 0);
+                const int y0 = (partial ? pc.slot : pc.b) * args.R + g * 128 + static_cast<int>(rank) * 64 +
+                               32 * (warp & 1);  // first of this warp's 32 rows
+                const int nblk = partial ? 8 : 4;  // fp32: 32 columns per box; bf16: 64
+#pragma unroll 1
+                for (int blk = 0; blk < nblk; ++blk) {
+                    const int i = partial ? (blk >> 2) : (blk >> 1);
+                    const int c0 = partial ? (blk & 3) * 32 : (blk & 1) * 64;
+                    uint32_t ra[32], rb[32];
+                    ptx::tmem_ld_32(lane_addr + 128 * i + c0, ra);
+                    if (!partial) ptx::tmem_ld_32(lane_addr + 128 * i + c0 + 32, rb);
+                    ptx::tmem_wait_ld();
+                    if (blk >= 2) {  // the store that last read this stage must be done with it
+                        if (lane == 0) ptx::bulk_wait_group_read<1>();
+                        __syncwarp();
+                    }
+                    uint8_t* sb = stage + (blk & 1) * 4096 + lane * 128;
+                    if (partial) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            *reinterpret_cast<float4*>(sb + ((k ^ (lane & 7)) << 4)) =
+                                make_float4(__uint_as_float(ra[4 * k + 0]) * inv_l, __uint_as_float(ra[4 * k + 1]) * inv_l,
+                                            __uint_as_float(ra[4 * k + 2]) * inv_l, __uint_as_float(ra[4 * k + 3]) * inv_l);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint32_t* src = (k < 4) ? (ra + 8 * k) : (rb + 8 * (k - 4));
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 bv = __floats2bfloat162_rn(__uint_as_float(src[2 * e]) * inv_l,
+                                                                                __uint_as_float(src[2 * e + 1]) * inv_l);
+                                w[e] = *reinterpret_cast<const uint32_t*>(&bv);
+                            }
+                            *reinterpret_cast<uint4*>(sb + ((k ^ (lane & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int col = 256 * i + 128 * h + c0;  // first value column of the box
+                        ptx::tma_store_2d(partial ? &tm_part : &tm_out, stage + (blk & 1) * 4096, col, y0);
+                        ptx::bulk_commit_group();
+                    }
+                }
+                if (lane == 0) ptx::bulk_wait_group_read<0>();  // stages free for the next piece's P
+                __syncwarp();
+            }
             ptx::tc_fence_before();
-            ok = group_barrier();  // sums buffer reused by the next piece
+            ok = group_barrier();  // sums buffer and P buffers reused by the next piece
         }
         if (!ok) atomicOr(args.status, kStatusTimeout);
+        // the output stores must be complete before this CTA's shared memory goes away
+        if (lane == 0) ptx::bulk_wait_group<0>();
+        __syncwarp();
     }
 
     // ---------------------------------------------------------------- teardown

@@ -133,13 +133,26 @@ constexpr int kDefaultSplitTiles = 16;  // batch-invariant chunks: 16 tiles = 20
 using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS, kPairNP>;
 
 mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                       const CUtensorMap& tm_v, const mla::MainArgs& args, cudaStream_t stream) {
+                       const CUtensorMap& tm_v, const CUtensorMap& tm_out, const CUtensorMap& tm_part,
+                       const mla::MainArgs& args, cudaStream_t stream) {
     auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV, kPairNS, kPairNP>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairC::kSmemBytes) != cudaSuccess)
         return MLA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(2 * plan.num_partitions * plan.num_groups));
-    kern<<<grid, PairC::kThreads, PairC::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, args);
+    kern<<<grid, PairC::kThreads, PairC::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_out, tm_part, args);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Output maps of the pair kernel's TMA-store epilogue: rows of 512 values,
+// boxes of 32 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle.
+bool encode_rows_store(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, bool fp32) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(mla::kDv), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(mla::kDv) * (fp32 ? 4 : 2)};
+    const cuuint32_t box[2] = {fp32 ? 32u : 64u, 32u};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 bool encode_2d_bf16(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
@@ -386,12 +399,16 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
     if (!enc) return MLA_ERR_CUDA;
 
     const int G = pl.group_rows;
-    CUtensorMap tm_q, tm_kv, tm_k;
+    CUtensorMap tm_q, tm_kv, tm_k, tm_out, tm_part;
     if (pl.kernel == MLA_KERNEL_PAIR) {
-        // Q: 64-row halves; K: 64 own kv rows per CTA; V: all 128 rows of a tile
+        // Q: 64-row halves; K: 64 own kv rows per CTA; V: all 128 rows of a tile;
+        // out and the fp32 partials: the epilogue's TMA stores
+        uint8_t* part_o = static_cast<uint8_t*>(workspace) + lay.part_o_off;
         if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, 64) ||
             !encode_kv(enc, &tm_k, kv, pl.L_max, pl.B, 64) ||
-            !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV))
+            !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV) ||
+            !encode_rows_store(enc, &tm_out, out, static_cast<uint64_t>(pl.B) * R, false) ||
+            !encode_rows_store(enc, &tm_part, part_o, static_cast<uint64_t>(num_slots(pl)) * R, true))
             return MLA_ERR_CUDA;
     } else if (fp8) {
         if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, G) ||
@@ -439,7 +456,7 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
     if (phases & 1) {
         mla_status st;
         if (pl.kernel == MLA_KERNEL_PAIR)
-            st = launch_pair(pl, tm_q, tm_k, tm_kv, a, stream);
+            st = launch_pair(pl, tm_q, tm_k, tm_kv, tm_out, tm_part, a, stream);
         else if (pl.kernel == MLA_KERNEL_FP8_MMA)
             st = (G == 16) ? launch_fp8mma<16>(pl, tm_kv, a, stream) : launch_fp8mma<32>(pl, tm_kv, a, stream);
         else if (fp8)
