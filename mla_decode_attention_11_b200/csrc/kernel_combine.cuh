@@ -49,14 +49,14 @@ constexpr int kCombineWarps = kCombineThreads / 32;
 // rows must be merged, never more than one per 8 rows.
 inline int combine_grid_y(int B, int R, int num_sms) {
     const int max_y = (R + kCombineWarps - 1) / kCombineWarps;
-    int y = (2 * num_sms + B - 1) / B;
+    int y = (2 * num_sms) / B;
     if (y < 1) y = 1;
     return y < max_y ? y : max_y;
 }
 
 // DV: value width (512 for MLA, 128 for MHA); a lane owns DV / 128 float4 columns.
 template <int DV = kDv>
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, 2)
     mla_decode_combine_kernel(const CombineArgs args) {
     static_assert(DV == 512 || DV == 128, "value width");
     constexpr int NV4 = DV / 128;  // float4 columns per lane
@@ -119,47 +119,31 @@ __global__ void __launch_bounds__(kCombineThreads)
         const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
         float4 acc_o[NV4];
         float lse_all;
-        if (k <= 4) {
-            // up to 4 pieces: every lane loads all their lse values and its
-            // columns of all their partial rows at once (one round trip)
-            float pl[4];
-            float4 x[4][NV4];
+        if (k <= 2) {
+            // two pieces (a sequence cut once, the common case): every lane loads
+            // both lse values and its columns of both partial rows at once (one
+            // round trip)
+            float pl[2];
+            float4 x[2][NV4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                pl[j] = -INFINITY;
-                if (j < k) {
-                    const size_t prow = static_cast<size_t>(slot_of(j)) * args.R + r;
-                    pl[j] = args.part_lse[prow];
-                    const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
+            for (int j = 0; j < 2; ++j) {
+                const size_t prow = static_cast<size_t>(slot_of(j)) * args.R + r;
+                pl[j] = args.part_lse[prow];
+                const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
 #pragma unroll
-                    for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
-                }
+                for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
             }
-            float m = sink;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) m = fmaxf(m, pl[j]);
-            float w[4], sum = expf(sink - m);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                w[j] = (j < k) ? expf(pl[j] - m) : 0.f;
-                sum += w[j];
-            }
+            const float m = fmaxf(fmaxf(pl[0], pl[1]), sink);
+            const float w0 = expf(pl[0] - m), w1 = expf(pl[1] - m);
+            const float sum = w0 + w1 + expf(sink - m);
             lse_all = m + logf(sum);
             const float inv = 1.f / sum;
 #pragma unroll
-            for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                if (j < k) {
-                    const float wj = w[j] * inv;
-#pragma unroll
-                    for (int v = 0; v < NV4; ++v) {
-                        acc_o[v].x += wj * x[j][v].x;
-                        acc_o[v].y += wj * x[j][v].y;
-                        acc_o[v].z += wj * x[j][v].z;
-                        acc_o[v].w += wj * x[j][v].w;
-                    }
-                }
+            for (int v = 0; v < NV4; ++v) {
+                acc_o[v].x = (w0 * inv) * x[0][v].x + (w1 * inv) * x[1][v].x;
+                acc_o[v].y = (w0 * inv) * x[0][v].y + (w1 * inv) * x[1][v].y;
+                acc_o[v].z = (w0 * inv) * x[0][v].z + (w1 * inv) * x[1][v].z;
+                acc_o[v].w = (w0 * inv) * x[0][v].w + (w1 * inv) * x[1][v].w;
             }
         } else {
             // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)

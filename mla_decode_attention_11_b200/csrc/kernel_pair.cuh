@@ -41,8 +41,11 @@
 // takes to execute, so the two GEMMs are issued from two threads.  A
 // cluster-scope release arrive costs a thread over a thousand cycles, so the
 // softmax warps only ever arrive at CTA scope: the follower's P-ready barrier
-// is forwarded to the leader by one otherwise idle thread.  Loads of both CTAs are counted on
-// the leader's barriers (2-SM TMA); MMA completion is multicast to both CTAs.
+// is forwarded to the leader by one otherwise idle thread, as a 4-byte
+// st.async into the leader's shared memory whose complete-tx (release at
+// cluster scope) lands on the leader's barrier; measured ~1,400 cycles sooner
+// than a release arrive.  Loads of both CTAs are counted on the leader's
+// barriers (2-SM TMA); MMA completion is multicast to both CTAs.
 // Every wait is bounded; on expiry a CTA records kStatusTimeout and unwinds.
 #pragma once
 
@@ -70,7 +73,8 @@ struct PairCfg {
     static constexpr int OFF_V = OFF_K + NK * kKChunk;
     static constexpr int OFF_P = OFF_V + NV * kVSlot;
     static constexpr int kPBuf = 2 * kPChunk;                 // one P tile (2 chunks of 64 keys)
-    static_assert(NP == 2, "two P buffers (they double as the 32 KB epilogue stage)");
+    static_assert(NP == 1 || NP == 2, "one or two P buffers (they double as the epilogue's store stages)");
+    static constexpr int kStagesPerWarp = NP;                 // 4 KB epilogue stages per softmax warp
     static constexpr int OFF_RED = OFF_P + NP * kPBuf;         // floats: [2][128] max, [128] sum
     static constexpr int OFF_BAR = OFF_RED + 384 * 4;
     // q_full, q_empty, pv_done[NP], drain_s, drain_pv, group_sync, s_full[NS], p_full[NS], p_local[NS],
@@ -81,6 +85,7 @@ struct PairCfg {
     static constexpr uint32_t kTmemCols = 512;                 // O: [0,256), S buffers from 256, 64 each
     static constexpr uint32_t kColS = 256;
     static_assert(NS >= 2 && 256 + 64 * NS <= 512, "S buffers must fit next to O in TMEM");
+    static_assert(NS <= 4, "one 4-byte forwarding slot per S buffer in the 64-byte misc area (words 12..15)");
     static constexpr uint32_t kIdescS = ptx::make_idesc_bf16(128, 128, 0, 0);
     static constexpr uint32_t kIdescPV = ptx::make_idesc_bf16(128, 256, 0, 1);
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -108,7 +113,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     uint64_t* group_sync = drain_pv + 1;
     uint64_t* s_full = group_sync + 1;      // [NS] S buffer b holds a finished QK^T
     uint64_t* p_full = s_full + NS;         // [NS] leader: the tile in S buffer b is through both softmaxes
-                                            //      (its S read, its P written in both CTAs)
+                                            //      (its S read, its P written in both CTAs): 128 arrivals
+                                            //      and 4 transaction bytes stored by the follower
     uint64_t* p_local = p_full + NS;        // [NS] follower: the same, for this CTA's 128 softmax threads
     uint64_t* k_full = p_local + NS;
     uint64_t* k_empty = k_full + NK;
@@ -120,6 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     long long* acc_first_slot = reinterpret_cast<long long*>(misc + 4);
     long long* total_slot = reinterpret_cast<long long*>(misc + 6);
     int* split_slot = reinterpret_cast<int*>(misc + 8);  // schedule chunk size of this run (0: balanced)
+    uint32_t* fwd_slot = misc + 12;                       // [NS] leader: target of the follower's P-ready store
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -138,7 +145,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         ptx::mbar_init(q_empty, 1);
         for (int i = 0; i < NS; ++i) {
             ptx::mbar_init(s_full + i, 1);
-            ptx::mbar_init(p_full + i, 129);   // leader's 128 softmax threads + the follower's forwarder
+            ptx::mbar_init(p_full + i, 128);   // leader's 128 softmax threads (+ 4 tx bytes from the follower)
             ptx::mbar_init(p_local + i, 128);  // follower's 128 softmax threads
         }
         for (int i = 0; i < NP; ++i) ptx::mbar_init(pv_done + i, 1);
@@ -285,13 +292,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             // before teardown, every load this CTA pair may still have in flight
             // must have landed: the leader counts both CTAs' bytes, so it waits
             // (bounded) for the last phase it armed on each K slot and on Q
+            // (a drain that runs out means a load never landed: recorded as a timeout)
             if (leader) {
+                bool drained = true;
                 const uint32_t n_k = k_cnt < static_cast<uint32_t>(NK) ? k_cnt : static_cast<uint32_t>(NK);
                 for (uint32_t i = 0; i < n_k; ++i) {
                     const uint32_t c = k_cnt - 1 - i;
-                    ptx::mbar_wait_bounded(k_full + c % NK, (c / NK) & 1, tmo);
+                    drained &= ptx::mbar_wait_bounded(k_full + c % NK, (c / NK) & 1, tmo);
                 }
-                if (piece_cnt > 0) ptx::mbar_wait_bounded(q_full, (piece_cnt - 1) & 1, tmo);
+                if (piece_cnt > 0) drained &= ptx::mbar_wait_bounded(q_full, (piece_cnt - 1) & 1, tmo);
+                if (!drained) atomicOr(args.status, kStatusTimeout);
             }
         }
         __syncwarp();
@@ -321,11 +331,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             }
             if (!ok) atomicOr(args.status, kStatusTimeout);
             if (leader) {  // as for K: the last armed phase of each V slot has landed
+                bool drained = true;
                 const uint32_t n_v = v_cnt < static_cast<uint32_t>(NV) ? v_cnt : static_cast<uint32_t>(NV);
                 for (uint32_t i = 0; i < n_v; ++i) {
                     const uint32_t c = v_cnt - 1 - i;
-                    ptx::mbar_wait_bounded(v_full + c % NV, (c / NV) & 1, tmo);
+                    drained &= ptx::mbar_wait_bounded(v_full + c % NV, (c / NV) & 1, tmo);
                 }
+                if (!drained) atomicOr(args.status, kStatusTimeout);
             }
         }
         __syncwarp();
@@ -385,7 +397,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         __syncwarp();
     } else if (warp == 7 && !leader) {
         // ============================================================ P-ready forwarder (follower)
-        // One cluster-scope release per tile, made here instead of by every softmax thread.
+        // One cluster-scope release per tile (the st.async's complete-tx), made here
+        // instead of by every softmax thread.
         if (ptx::elect_one()) {
             bool ok = true;
             uint32_t u = 0;
@@ -394,7 +407,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 for (int t = pc.tile_lo; ok && t < pc.tile_hi; ++t, ++u) {
                     const uint32_t b = u % NS;
                     ok = ptx::mbar_wait_bounded(p_local + b, (u / NS) & 1, tmo);
-                    if (ok) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(p_full + b), 0));
+                    // a 4-byte st.async into the leader's fwd slot, counted on its p_full
+                    if (ok)
+                        ptx::st_async_u32(ptx::mapa_shared(ptx::smem_u32(fwd_slot + b), 0), u,
+                                          ptx::mapa_shared(ptx::smem_u32(p_full + b), 0));
                 }
             }
             if (!ok) atomicOr(args.status, kStatusTimeout);
@@ -589,7 +605,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
                 // CTA-scope arrive: the leader's own barrier, or the follower's local one
-                ptx::mbar_arrive(leader ? (p_full + buf) : (p_local + buf));
+                // (the leader's thread 0 also arms the 4 bytes the follower's forwarder stores)
+                if (leader && L_id == 0) ptx::mbar_arrive_expect_tx(p_full + buf, 4);
+                else ptx::mbar_arrive(leader ? (p_full + buf) : (p_local + buf));
                 ++tile_cnt;
             }
             if (!ok) break;
@@ -623,11 +641,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             // 32 rows x 128 bytes are written into a 4 KB stage in the 128-byte
             // swizzle a TMA store expects (lane = row, so each instruction
             // spreads over all banks), and one lane stores the box with TMA.
-            // Each warp owns 8 KB of the P buffers (two stages, alternating):
+            // Each warp owns NP 4 KB stages of the P buffers, used in turn:
             // every PV of the piece has completed, and the next piece's P is
             // written only after the closing group barrier.
             {
-                uint8_t* stage = p_smem + warp * 8192;
+                constexpr int NST = C::kStagesPerWarp;
+                uint8_t* stage = p_smem + warp * (NST * 4096);
                 const bool partial = (pc.slot >= 0);
                 const int y0 = (partial ? pc.slot : pc.b) * args.R + g * 128 + static_cast<int>(rank) * 64 +
                                32 * (warp & 1);  // first of this warp's 32 rows
@@ -640,11 +659,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                     ptx::tmem_ld_32(lane_addr + 128 * i + c0, ra);
                     if (!partial) ptx::tmem_ld_32(lane_addr + 128 * i + c0 + 32, rb);
                     ptx::tmem_wait_ld();
-                    if (blk >= 2) {  // the store that last read this stage must be done with it
-                        if (lane == 0) ptx::bulk_wait_group_read<1>();
+                    if (blk >= NST) {  // the store that last read this stage must be done with it
+                        if (lane == 0) ptx::bulk_wait_group_read<NST - 1>();
                         __syncwarp();
                     }
-                    uint8_t* sb = stage + (blk & 1) * 4096 + lane * 128;
+                    uint8_t* sb = stage + (blk % NST) * 4096 + lane * 128;
                     if (partial) {
 #pragma unroll
                         for (int k = 0; k < 8; ++k)
@@ -669,7 +688,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                     __syncwarp();
                     if (lane == 0) {
                         const int col = 256 * i + 128 * h + c0;  // first value column of the box
-                        ptx::tma_store_2d(partial ? &tm_part : &tm_out, stage + (blk & 1) * 4096, col, y0);
+                        ptx::tma_store_2d(partial ? &tm_part : &tm_out, stage + (blk % NST) * 4096, col, y0);
                         ptx::bulk_commit_group();
                     }
                 }

@@ -249,6 +249,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// 4-byte asynchronous store into shared memory of a CTA of this cluster whose
+// completion is counted as 4 transaction bytes on an mbarrier there; the
+// complete-tx has release semantics at cluster scope, so everything this
+// thread has observed before it is visible to a cluster-scope acquire of that
+// barrier's phase (a cheaper signal than a cluster-scope release arrive).
+__device__ __forceinline__ void st_async_u32(uint32_t cluster_addr, uint32_t v, uint32_t bar_cluster_addr) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr),
+                 "r"(v), "r"(bar_cluster_addr)
+                 : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

@@ -199,17 +199,20 @@ def test_seqlen_out_of_range_is_flagged(cuda_device):
     M.mla_decode_check(plan, ws)  # cleared after the read
 
 
-@pytest.mark.parametrize("H", [16, 128])
-def test_bounded_wait_timeout_reports_and_recovers(cuda_device, H):
+@pytest.mark.parametrize("H,unit,parts", [(16, 3, 0), (128, 3, 0), (16, 30, 1), (128, 40, 1)])
+def test_bounded_wait_timeout_reports_and_recovers(cuda_device, H, unit, parts):
     """A host-side fault injection: the producer of CTA 0 arms a barrier but
-    skips the load, so the consumer's bounded wait runs out.  The run must
-    report MLA_ERR_TIMEOUT, and the context must stay usable."""
+    skips a load (an early one, or one deep in the stream with several loads
+    of both CTAs still in flight), so the consumer's bounded wait runs out and
+    every role unwinds, draining what it armed.  The run must report
+    MLA_ERR_TIMEOUT, and the context must stay usable."""
     w = W.custom(B=2, Sq=1, H=H, L=1000, seed=101)
     q, kv, sl = W.generate(w)
     try:
-        M.mla_decode_set_debug(wait_timeout_ns=20_000_000, stall_unit=3)
+        M.mla_decode_set_debug(wait_timeout_ns=20_000_000, stall_unit=unit)
         dev = torch.device("cuda:0")
-        plan = M.mla_decode_plan(2, 1, H, 1000, device=0)
+        # one partition: CTA 0 streams all 16 tiles, so a late unit lies mid-stream
+        plan = M.mla_decode_plan(2, 1, H, 1000, device=0, num_partitions=parts)
         ws = M.alloc_workspace(plan)
         out = torch.empty((2, 1, H, 512), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((2, 1, H), dtype=torch.float32, device=dev)
@@ -224,7 +227,7 @@ def test_bounded_wait_timeout_reports_and_recovers(cuda_device, H):
     M.mla_decode_run(plan, q.to(dev), kv.to(dev), sl.to(dev), w.scale, out, lse, ws)
     M.mla_decode_check(plan, ws)
     ro, rl = oracle.mla_decode(q, kv, sl, w.scale)
-    assert_parity(out.cpu(), lse.cpu(), ro, rl, f"after timeout H{H}")
+    assert_parity(out.cpu(), lse.cpu(), ro, rl, f"after timeout H{H} unit {unit}")
     check_workload(w)
 
 
