@@ -604,7 +604,7 @@ def run_fp8(args, w: W.Workload):
     torch.cuda.set_device(dev)
     q, codes, ks, sl = W.generate_fp8(w)
     qd, cd, sld = q.to(dev), codes.to(dev), sl.to(dev)
-    kernel = M.MLA_KERNEL_FP8
+    kernel = M.MLA_KERNEL_FP8 if args.fp8_kernel == "widen" else M.MLA_KERNEL_FP8_MMA
     plan = M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=0, kernel=kernel)
     ws = M.alloc_workspace(plan, device=dev)
     M.mla_decode_workspace_init(plan, ws)
@@ -737,6 +737,8 @@ def main():
                     help="time the attention-sink entry point (per-head sink logits) on the same workload")
     ap.add_argument("--fp8", action="store_true",
                     help="the same MLA workload over an FP8 (E4M3) latent cache (mla_decode_run_fp8)")
+    ap.add_argument("--fp8-kernel", choices=["operands", "widen"], default="operands",
+                    help="FP8 cache kernel: codes as kind::f8f6f4 MMA operands (default) or widened to f16")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -66,7 +66,7 @@ enum {
     MLA_KERNEL_FP8 = 4,        /* MLA decode over an FP8 cache (mla_decode_plan_fp8): the transposed kernel
                                   with E4M3 chunks widened to f16 in shared memory */
     MLA_KERNEL_FP8_MMA = 5     /* MLA decode over an FP8 cache with the codes as kind::f8f6f4 MMA operands
-                                  (mla_decode_plan_fp8_kernel); experimental, see there */
+                                  (what mla_decode_plan_fp8 picks; see mla_decode_plan_fp8_kernel) */
 };
 
 /*
@@ -339,31 +339,31 @@ mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void*
  * at the top of this file on those values (keys: all 576 columns; values:
  * the first 512), with q bf16, out bf16 and lse fp32 as there.
  *
- * Numerics: every E4M3 value divided by 2^8 is exact in f16, so the kernel
- * widens the codes to those f16 values in shared memory (integer bit moves)
- * and runs f16 x f16 -> f32 tensor-core MMAs; q is narrowed from bf16 to f16
- * (exact for 2^-17 <= |q| <= 65504; |q| > 65504 becomes inf, smaller |q| lose
- * at most 2^-25), P is rounded to f16, and kv_scale * 2^8 multiplies the
- * scores (with softmax_scale) and the output rows.
+ * Numerics, by kernel (both keep the cache's values exact and accumulate in fp32):
+ *   MLA_KERNEL_FP8_MMA (the default): the codes are the operands of
+ *     kind::f8f6f4 tensor-core MMAs as they are; each q row is scaled by a
+ *     power of two and carried as the sum of three E4M3 terms (about 12
+ *     significant bits, relative error <= 2^-12), and P (scaled by 2^7) as the
+ *     sum of two (about 8 bits, the precision of the bf16 P of the bf16 path).
+ *   MLA_KERNEL_FP8: every E4M3 value divided by 2^8 is exact in f16, so the
+ *     kernel widens the codes to those f16 values in shared memory (integer
+ *     bit moves) and runs f16 x f16 -> f32 MMAs; q is narrowed from bf16 to f16
+ *     (exact for 2^-17 <= |q| <= 65504; |q| > 65504 becomes inf, smaller |q|
+ *     lose at most 2^-25), P is rounded to f16, and kv_scale * 2^8 multiplies
+ *     the scores (with softmax_scale) and the output rows.
  *
  * mla_decode_plan_fp8 -- as mla_decode_plan (same arguments, limits and return
- * codes) for an FP8 cache; the plan's kernel is MLA_KERNEL_FP8 (the transposed
- * kernel, 16 or 32 query rows per CTA, 320 threads), for every head count.
+ * codes) for an FP8 cache; the plan's kernel is MLA_KERNEL_FP8_MMA (16 or 32
+ * query rows per CTA, 192 threads), for every head count.
  */
 mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
                                int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
 
 /*
  * mla_decode_plan_fp8_kernel -- mla_decode_plan_fp8 with an explicit kernel:
- *   kernel  0 or MLA_KERNEL_FP8: the widening kernel (what mla_decode_plan_fp8 picks);
- *           MLA_KERNEL_FP8_MMA: EXPERIMENTAL -- the codes are the operands of
- *           kind::f8f6f4 MMAs and q and P are carried as sums of E4M3 terms (q:
- *           three terms of a power-of-two-scaled row, about 12 significant bits;
- *           P: two terms, about 8), so its results differ from the exact-operand
- *           path by those truncations.  Only a library built with
- *           MLA_EXPERIMENTAL_FP8MMA defined plans it; otherwise this kernel
- *           returns MLA_ERR_UNSUPPORTED (from the plan, and from a run given a
- *           plan of this kind).
+ *   kernel  0 or MLA_KERNEL_FP8_MMA: the codes as MMA operands (what
+ *           mla_decode_plan_fp8 picks; q and P carried as sums of E4M3 terms);
+ *           MLA_KERNEL_FP8: the widening kernel (f16 operands, 320 threads).
  *           Anything else: MLA_ERR_INVALID_ARG.
  * Other arguments and return codes as mla_decode_plan_fp8; the plan runs
  * through mla_decode_run_fp8.
@@ -384,8 +384,9 @@ mla_status mla_decode_plan_fp8_kernel(int32_t B, int32_t Sq, int32_t H, int32_t 
  *            as mla_decode_run;  sinks as mla_decode_run_sinks (NULL = none)
  * Launches the main kernel and the split-KV combine; no host sync, no
  * allocation; return codes as mla_decode_run.  The cache must hold finite
- * codes: the two NaN codes (S.1111.111) are read as +-480 (times kv_scale),
- * not as NaN.
+ * codes (a quantiser saturates): a NaN code (S.1111.111) in a used row gives
+ * unspecified results (NaN with MLA_KERNEL_FP8_MMA, +-480 * kv_scale with
+ * MLA_KERNEL_FP8).
  */
 mla_status mla_decode_run_fp8(const mla_plan* plan, const void* q, const void* kv_fp8, float kv_scale,
                               const int32_t* seqlens, float softmax_scale, const float* sinks, void* out, float* lse,

@@ -126,10 +126,10 @@ def test_batch_invariant_plan_without_gpu():
 
 
 def test_fp8_plan_without_gpu():
-    p = M.mla_decode_plan_fp8(132, 1, 16, 16384, device=-1)
+    p = M.mla_decode_plan_fp8(132, 1, 16, 16384, device=-1, kernel=M.MLA_KERNEL_FP8)
     assert p.kernel == M.MLA_KERNEL_FP8 and p.group_rows == 16 and p.cta_threads == 320
     assert p.num_partitions == 148 and p.smem_bytes <= 232448
-    p = M.mla_decode_plan_fp8(64, 1, 128, 8192, device=-1)
+    p = M.mla_decode_plan_fp8(64, 1, 128, 8192, device=-1, kernel=M.MLA_KERNEL_FP8)
     assert p.kernel == M.MLA_KERNEL_FP8 and p.group_rows == 32 and p.num_groups == 4 and p.cta_threads == 256
     assert p.workspace_bytes == M.mla_decode_plan(64, 1, 128, 8192, device=-1,
                                                   kernel=M.MLA_KERNEL_TRANSPOSED).workspace_bytes
@@ -165,23 +165,14 @@ def test_fp8_run_rejects_without_launching(lib):
 
 
 def test_fp8_operand_kernel_plan_without_gpu():
-    """The FP8-operand kernel is not offered by the default build (it has not
-    matched the oracle on a GPU yet): an explicit request is refused as
-    unsupported, and the automatic choice is the widening kernel."""
-    assert M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1).kernel == M.MLA_KERNEL_FP8
-    for H in (16, 128):
-        with pytest.raises(M.MlaError) as e:
-            M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8_MMA)
-        assert e.value.code == 3
-    # a hand-made plan of that kind is refused by the run entry point before
-    # anything touches a device
-    lib = M.load_library()
-    f8 = M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1)
-    f8.kernel = M.MLA_KERNEL_FP8_MMA
-    sc = ctypes.c_float(576 ** -0.5)
-    rc = lib.mla_decode_run_fp8(ctypes.byref(f8), 16, 16, ctypes.c_float(0.5), 16, sc, None, 16, 16, 256,
-                                f8.workspace_bytes, None)
-    assert rc == 3
+    """The FP8-operand kernel is the default FP8 plan; the widening kernel is
+    chosen explicitly; other kinds are refused."""
+    for H, G in ((16, 16), (128, 32)):
+        p = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1)
+        assert p.kernel == M.MLA_KERNEL_FP8_MMA and p.group_rows == G and p.cta_threads == 192
+        assert p.smem_bytes <= 232448
+        w = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8)
+        assert w.kernel == M.MLA_KERNEL_FP8 and w.group_rows == G
     for bad in (1, 2, 3, 6):
         with pytest.raises(M.MlaError) as e:
             M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1, kernel=bad)
