@@ -71,20 +71,20 @@ struct Fp8MmaCfg {
     static constexpr int OFF_PAIR = 0;
     static constexpr int OFF_ROPE = OFF_PAIR + NP * kPairBytes;
     static constexpr int OFF_Q = OFF_ROPE + NR * kChunkBytes;
-    static constexpr int OFF_P = OFF_Q + kNumChunks * kQChunkBytes;
-    static constexpr int OFF_QS = OFF_P + kPBytes;                 // G floats
+    static constexpr int OFF_P = OFF_Q + kNumChunks * kQChunkBytes;  // two P buffers (tiles alternate)
+    static constexpr int OFF_QS = OFF_P + 2 * kPBytes;             // G floats
     static constexpr int OFF_RED = OFF_QS + G * 4;                 // floats: [2][4][G] max, [4][G] sums
     static constexpr int kRedFloats = 12 * G;
     static constexpr int OFF_BAR = OFF_RED + kRedFloats * 4;
-    // barriers: q_ready, q_empty, s_full, p_full, pv_done, drain, group_sync,
+    // barriers: q_ready, q_empty, s_full[2], p_full[2], pv_tile[2], pv_done, drain, group_sync,
     //           pair_full[NP], pair_empty[NP], rope_full[NR], rope_empty[NR]
-    static constexpr int kNumBars = 7 + 2 * NP + 2 * NR;
+    static constexpr int kNumBars = 11 + 2 * NP + 2 * NR;
     static constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
     static constexpr int kSmemBytes = OFF_MISC + 64 + 1024;
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(OFF_Q % 1024 == 0 && OFF_P % 1024 == 0, "swizzled regions start on 1024-byte boundaries");
-    // TMEM: O^T blocks at columns [0, 4 NO), S^T after them
-    static constexpr int kCols = 4 * NO + NS;
+    // TMEM: O^T blocks at columns [0, 4 NO), then two S^T buffers (tiles alternate)
+    static constexpr int kCols = 4 * NO + 2 * NS;
     static constexpr uint32_t kTmemCols = kCols <= 256 ? 256 : 512;
     static constexpr uint32_t kColS = 4 * NO;
     // P^T rows are 2G codes = 32 or 64 bytes
@@ -148,12 +148,13 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* q_ready = bars + 0;     // the softmax threads wrote this piece's Q terms
     uint64_t* q_empty = bars + 1;     // the piece's last S^T MMA completed
-    uint64_t* s_full = bars + 2;
-    uint64_t* p_full = bars + 3;
-    uint64_t* pv_done = bars + 4;
-    uint64_t* drain = bars + 5;
-    uint64_t* group_sync = bars + 6;  // the 128 softmax threads (bounded, unlike bar.sync)
-    uint64_t* pair_full = bars + 7;
+    uint64_t* s_full = bars + 2;      // [2] S^T buffer b holds a finished QK^T (tiles alternate)
+    uint64_t* p_full = bars + 4;      // [2] P buffer b written by the 128 softmax threads
+    uint64_t* pv_tile = bars + 6;     // [2] the PV that read P buffer b has completed
+    uint64_t* pv_done = bars + 8;     // the piece's last PV has completed
+    uint64_t* drain = bars + 9;
+    uint64_t* group_sync = bars + 10; // the 128 softmax threads (bounded, unlike bar.sync)
+    uint64_t* pair_full = bars + 11;
     uint64_t* pair_empty = pair_full + C::NP;
     uint64_t* rope_full = pair_empty + C::NP;
     uint64_t* rope_empty = rope_full + C::NR;
@@ -174,8 +175,11 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         ptx::mbar_init(q_ready, 128);
         ptx::mbar_init(q_empty, 1);
-        ptx::mbar_init(s_full, 1);
-        ptx::mbar_init(p_full, 128);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(s_full + b, 1);
+            ptx::mbar_init(p_full + b, 128);
+            ptx::mbar_init(pv_tile + b, 1);
+        }
         ptx::mbar_init(pv_done, 1);
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(group_sync, 128);
@@ -314,68 +318,83 @@ __global__ void __launch_bounds__(192, 1)
     } else if (warp == 5) {
 
         // ============================================================ MMA issuer
+        // Within a piece, QK^T of tile t+1 goes to the tensor pipe before the
+        // issuer waits for tile t's softmax, so the pipe works on the next S^T
+        // while the softmax runs; S^T and P are double-buffered by tile parity.
+        // Pipe order per piece: S(0), S(1), PV(0), S(2), PV(1), ..., PV(last):
+        // S(t+2) follows PV(t), so when the softmax sees S(t+2) complete, PV(t)
+        // has stopped reading P buffer t % 2 and S^T buffer t % 2 is free again.
+        // Not across pieces: the next piece's Q terms are written by the softmax
+        // threads after this piece's epilogue, which waits for the last PV.
         if (ptx::elect_one()) {
             uint32_t pair_cnt = 0, rope_cnt = 0, piece_cnt = 0, tile_cnt = 0;
             bool ok = true;
             const uint32_t q_base = ptx::smem_u32(q_smem);
-            const uint32_t p_base = ptx::smem_u32(p_smem);
-            const uint32_t tm_S = tmem_base + C::kColS;
+            const uint32_t p_base0 = ptx::smem_u32(p_smem);
+            uint32_t slots[2][4];  // the pair slots of the tiles in flight, by tile parity
+            // S^T(t) = K . [Q1 Q2 Q3]^T for global tile index u (rope chunk first, then the 8 value chunks)
+            auto issue_qk = [&](uint32_t u, bool last) -> bool {
+                const uint32_t sb = u & 1;
+                const uint32_t tm_S = tmem_base + C::kColS + sb * C::NS;
+                const uint32_t rs = rope_cnt % C::NR;
+                if (!ptx::mbar_wait_bounded(rope_full + rs, (rope_cnt / C::NR) & 1, tmo)) return false;
+                ptx::tc_fence_after();
+                {
+                    const uint32_t a0 = ptx::smem_u32(rope_smem + rs * C::kChunkBytes);
+                    const uint32_t b0 = q_base + (kNumChunks - 1) * C::kQChunkBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {  // 32 codes = 32 bytes per MMA
+                        const uint64_t da = ptx::make_smem_desc(a0 + kk * 32, 16, 512, ptx::Swizzle::B64);
+                        const uint64_t db = ptx::make_smem_desc(b0 + kk * 32, 16, 512, ptx::Swizzle::B64);
+                        mma_e4m3_ss(tm_S, da, db, C::kIdescS, kk > 0 ? 1u : 0u);
+                    }
+                }
+                ptx::mma_commit(rope_empty + rs);
+                ++rope_cnt;
+                for (int pp = 0; pp < 4; ++pp) {
+                    const uint32_t s = (pair_cnt + pp) % C::NP;
+                    slots[sb][pp] = s;
+                    if (!ptx::mbar_wait_bounded(pair_full + s, ((pair_cnt + pp) / C::NP) & 1, tmo)) return false;
+                    ptx::tc_fence_after();
+                    const uint32_t pbase = ptx::smem_u32(pair_smem + s * C::kPairBytes);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int c = 2 * pp + h;
+#pragma unroll
+                        for (int kk = 0; kk < 2; ++kk) {
+                            const uint64_t da = ptx::make_smem_desc(pbase + h * C::kChunkBytes + kk * 32, 16,
+                                                                    512, ptx::Swizzle::B64);
+                            const uint64_t db = ptx::make_smem_desc(q_base + c * C::kQChunkBytes + kk * 32, 16,
+                                                                    512, ptx::Swizzle::B64);
+                            mma_e4m3_ss(tm_S, da, db, C::kIdescS, 1u);
+                        }
+                    }
+                }
+                pair_cnt += 4;
+                if (last) ptx::mma_commit(q_empty);
+                ptx::mma_commit(s_full + sb);
+                return true;
+            };
             Piece pc;
             while (ok && walker.next(pc)) {
-                for (int t = pc.tile_lo; t < pc.tile_hi; ++t) {
-                    const bool first = (t == pc.tile_lo);
-                    const bool last = (t == pc.tile_hi - 1);
-                    if (first) {
-                        ok = ptx::mbar_wait_bounded(q_ready, piece_cnt & 1, tmo);
+                ok = ptx::mbar_wait_bounded(q_ready, piece_cnt & 1, tmo);
+                if (!ok) break;
+                const int n = pc.tile_hi - pc.tile_lo;
+                ok = issue_qk(tile_cnt, n == 1);
+                for (int i = 0; ok && i < n; ++i) {
+                    const uint32_t u = tile_cnt;
+                    if (i + 1 < n) {
+                        ok = issue_qk(u + 1, i + 2 == n);
                         if (!ok) break;
                     }
-                    // ---------------- S^T = K . [Q1 Q2 Q3]^T  (rope chunk first, then the 8 value chunks)
-                    const uint32_t rs = rope_cnt % C::NR;
-                    ok = ptx::mbar_wait_bounded(rope_full + rs, (rope_cnt / C::NR) & 1, tmo);
+                    // ---------------- O^T += V^T . [P1 P2]^T  (after the softmax wrote tile u's P terms)
+                    const uint32_t pb = u & 1;
+                    ok = ptx::mbar_wait_bounded(p_full + pb, (u >> 1) & 1, tmo);
                     if (!ok) break;
                     ptx::tc_fence_after();
-                    {
-                        const uint32_t a0 = ptx::smem_u32(rope_smem + rs * C::kChunkBytes);
-                        const uint32_t b0 = q_base + (kNumChunks - 1) * C::kQChunkBytes;
-#pragma unroll
-                        for (int kk = 0; kk < 2; ++kk) {  // 32 codes = 32 bytes per MMA
-                            const uint64_t da = ptx::make_smem_desc(a0 + kk * 32, 16, 512, ptx::Swizzle::B64);
-                            const uint64_t db = ptx::make_smem_desc(b0 + kk * 32, 16, 512, ptx::Swizzle::B64);
-                            mma_e4m3_ss(tm_S, da, db, C::kIdescS, kk > 0 ? 1u : 0u);
-                        }
-                    }
-                    ptx::mma_commit(rope_empty + rs);
-                    ++rope_cnt;
-                    uint32_t slots[4];
+                    const uint32_t p_base = p_base0 + pb * C::kPBytes;
                     for (int pp = 0; pp < 4; ++pp) {
-                        const uint32_t s = (pair_cnt + pp) % C::NP;
-                        slots[pp] = s;
-                        ok = ptx::mbar_wait_bounded(pair_full + s, ((pair_cnt + pp) / C::NP) & 1, tmo);
-                        if (!ok) break;
-                        ptx::tc_fence_after();
-                        const uint32_t pbase = ptx::smem_u32(pair_smem + s * C::kPairBytes);
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int c = 2 * pp + h;
-#pragma unroll
-                            for (int kk = 0; kk < 2; ++kk) {
-                                const uint64_t da = ptx::make_smem_desc(pbase + h * C::kChunkBytes + kk * 32, 16,
-                                                                        512, ptx::Swizzle::B64);
-                                const uint64_t db = ptx::make_smem_desc(q_base + c * C::kQChunkBytes + kk * 32, 16,
-                                                                        512, ptx::Swizzle::B64);
-                                mma_e4m3_ss(tm_S, da, db, C::kIdescS, 1u);
-                            }
-                        }
-                    }
-                    if (!ok) break;
-                    if (last) ptx::mma_commit(q_empty);
-                    ptx::mma_commit(s_full);
-                    // ---------------- O^T += V^T . [P1 P2]^T  (after the softmax wrote the P terms)
-                    ok = ptx::mbar_wait_bounded(p_full, tile_cnt & 1, tmo);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    for (int pp = 0; pp < 4; ++pp) {
-                        const uint32_t vbase = ptx::smem_u32(pair_smem + slots[pp] * C::kPairBytes);
+                        const uint32_t vbase = ptx::smem_u32(pair_smem + slots[pb][pp] * C::kPairBytes);
                         const uint32_t tm_O = tmem_base + pp * C::NO;
 #pragma unroll
                         for (int kk = 0; kk < kTileKV / 32; ++kk) {
@@ -386,12 +405,12 @@ __global__ void __launch_bounds__(192, 1)
                             // B = the P terms: K = 32 kv rows (four atoms), N = 2G (one atom wide)
                             const uint64_t db = ptx::make_smem_desc(p_base + kk * 4 * C::kPAtom, C::kPBytes,
                                                                     C::kPAtom, C::kPSwz);
-                            mma_e4m3_ss(tm_O, da, db, C::kIdescPV, (!first || kk > 0) ? 1u : 0u);
+                            mma_e4m3_ss(tm_O, da, db, C::kIdescPV, (i > 0 || kk > 0) ? 1u : 0u);
                         }
-                        ptx::mma_commit(pair_empty + slots[pp]);
+                        ptx::mma_commit(pair_empty + slots[pb][pp]);
                     }
-                    pair_cnt += 4;
-                    if (last) ptx::mma_commit(pv_done);
+                    ptx::mma_commit(pv_tile + pb);
+                    if (i + 1 == n) ptx::mma_commit(pv_done);
                     ++tile_cnt;
                 }
                 ++piece_cnt;
@@ -505,21 +524,23 @@ __global__ void __launch_bounds__(192, 1)
                 const int kv_row = row0 + row_in_tile;
                 const bool valid = (kv_row >= t * kTileKV) && (kv_row < pc.L);
 
-                ok = ptx::mbar_wait_bounded(s_full, tile_cnt & 1, tmo);
+                const uint32_t sb = tile_cnt & 1;  // S^T and P buffer of this tile
+                ok = ptx::mbar_wait_bounded(s_full + sb, (tile_cnt >> 1) & 1, tmo);
                 if (!ok) break;
                 ptx::tc_fence_after();
+                const uint32_t col_s = C::kColS + sb * C::NS;
                 float x[G];
 #pragma unroll
                 for (int c0 = 0; c0 < G; c0 += 16) {
                     uint32_t r[16];
                     float acc[16];
-                    ptx::tmem_ld_16(lane_addr + C::kColS + c0, r);
+                    ptx::tmem_ld_16(lane_addr + col_s + c0, r);
                     ptx::tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) acc[j] = __uint_as_float(r[j]);
 #pragma unroll
                     for (int k = 1; k < C::kQTerms; ++k) {
-                        ptx::tmem_ld_16(lane_addr + C::kColS + k * G + c0, r);
+                        ptx::tmem_ld_16(lane_addr + col_s + k * G + c0, r);
                         ptx::tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 16; ++j) acc[j] += __uint_as_float(r[j]);
@@ -553,6 +574,11 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int j = 0; j < G; ++j) m_ref[j] = tmax[j];
                 } else if (grow) {
+                    // O^T must hold the previous tile's PV before it is rescaled (this
+                    // tile's PV waits for the P written below)
+                    ok = ptx::mbar_wait_bounded(pv_tile + ((tile_cnt - 1) & 1), ((tile_cnt - 1) >> 1) & 1, tmo);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
                     float alpha[G];
 #pragma unroll
                     for (int j = 0; j < G; ++j) {
@@ -577,7 +603,10 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     ptx::tmem_wait_st();
                 }
-                // P terms of this kv row: 2^7 p = t1 + t2 (E4M3), t1 in bytes [0, G), t2 in [G, 2G)
+                // P terms of this kv row: 2^7 p = t1 + t2 (E4M3), t1 in bytes [0, G), t2 in [G, 2G);
+                // P buffer sb was last read by the PV of tile - 2, which the tensor pipe ran
+                // before this tile's S^T
+                uint8_t* p_buf = p_smem + sb * C::kPBytes;
                 uint32_t w1[G / 4], w2[G / 4];
 #pragma unroll
                 for (int j = 0; j < G; j += 2) {
@@ -599,14 +628,14 @@ __global__ void __launch_bounds__(192, 1)
                 }
 #pragma unroll
                 for (int u = 0; u < kUnitsPerTerm; ++u) {
-                    *reinterpret_cast<uint4*>(p_smem + swz_offset(row_in_tile, u, C::NO)) =
+                    *reinterpret_cast<uint4*>(p_buf + swz_offset(row_in_tile, u, C::NO)) =
                         make_uint4(w1[4 * u], w1[4 * u + 1], w1[4 * u + 2], w1[4 * u + 3]);
-                    *reinterpret_cast<uint4*>(p_smem + swz_offset(row_in_tile, kUnitsPerTerm + u, C::NO)) =
+                    *reinterpret_cast<uint4*>(p_buf + swz_offset(row_in_tile, kUnitsPerTerm + u, C::NO)) =
                         make_uint4(w2[4 * u], w2[4 * u + 1], w2[4 * u + 2], w2[4 * u + 3]);
                 }
                 ptx::fence_proxy_async_smem();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(p_full);
+                ptx::mbar_arrive(p_full + sb);
                 ++tile_cnt;
             }
             if (!ok) break;
