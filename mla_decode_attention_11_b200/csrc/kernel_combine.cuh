@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
 #include "schedule.cuh"
 
 namespace mla {
@@ -77,6 +78,9 @@ __global__ void __launch_bounds__(kCombineThreads, 2)
         }
     }
     __syncthreads();
+    // launched as a programmatic dependent of the main kernel: the scan above
+    // reads only the lengths; partials and outputs wait for the main grid
+    ptx::wait_prior_grid();
     const int S = s_split;
     const long long acc = s_acc, tot = s_tot;
     const int rows_per = (args.R + static_cast<int>(gridDim.y) - 1) / static_cast<int>(gridDim.y);

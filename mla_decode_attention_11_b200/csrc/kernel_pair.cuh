@@ -196,6 +196,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     ptx::cluster_sync_all();  // peer barriers initialised before any cross-CTA signal
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
+    // the split-KV combine (launched after this kernel as a programmatic
+    // dependent) may start scheduling its CTAs; it waits for this grid's results
+    ptx::launch_dependents();
 
     PieceWalker walker;
     {

@@ -406,6 +406,9 @@ __global__ void __launch_bounds__(TransposedCfg<G, SH>::kThreads, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
+    // the split-KV combine (launched after this kernel as a programmatic
+    // dependent) may start scheduling its CTAs; it waits for this grid's results
+    ptx::launch_dependents();
 
     PieceWalker walker;
     {

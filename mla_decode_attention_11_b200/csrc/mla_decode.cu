@@ -148,6 +148,28 @@ bool encode_rows_store(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint
                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The combine kernel is a programmatic dependent of the main kernel before it
+// on the stream: its CTAs may start (and scan the lengths) while the main
+// kernel finishes, and wait in the kernel for the main grid's results.
+template <int DV>
+mla_status launch_combine(dim3 grid, const mla::CombineArgs& c, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(mla::kCombineThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mla::mla_decode_combine_kernel<DV>, c) != cudaSuccess) {
+        cudaGetLastError();
+        return MLA_ERR_CUDA;
+    }
+    return MLA_OK;
+}
+
 bool encode_2d_bf16(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                     uint32_t box_inner, uint32_t box_rows) {
     const cuuint64_t dims[2] = {inner, rows};
@@ -477,9 +499,7 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
     c.H = pl.H;
     c.split_tiles = pl.split_tiles;
     const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>(mla::combine_grid_y(pl.B, R, pl.num_sms)));
-    mla::mla_decode_combine_kernel<mla::kDv><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    return MLA_OK;
+    return launch_combine<mla::kDv>(cgrid, c, stream);
 }
 
 mla_status run_phases(const mla_plan* plan, const void* q, const void* kv, const int32_t* seqlens,
@@ -820,9 +840,7 @@ mla_status mha_run_phases(const mla_plan* plan, const void* q, const void* k, co
     c.H = pl.H;
     c.split_tiles = pl.split_tiles;
     const dim3 cgrid(static_cast<unsigned>(pl.B), static_cast<unsigned>(mla::combine_grid_y(pl.B, R, pl.num_sms)));
-    mla::mla_decode_combine_kernel<kMhaD><<<cgrid, mla::kCombineThreads, 0, stream>>>(c);
-    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
-    return MLA_OK;
+    return launch_combine<kMhaD>(cgrid, c, stream);
 }
 
 }  // namespace
