@@ -40,9 +40,9 @@ struct CombineArgs {
 // lengths once (schedule and b's unit offset in one pass), so a sequence that
 // was not cut costs its CTAs one scan and nothing else; Y is chosen by the
 // host so that about two CTAs per SM share the merging of cut sequences.
-// Within a row the kernel is bound by the bytes of the partials it reads, so
-// each lane keeps up to 4 partials x 4 float4 in flight instead of walking the
-// partials one after another.
+// Within a row the kernel is bound by the latency of the partials it reads, so
+// each lane keeps up to 4 partials x 4 float4 in flight, requested before the
+// merged lse is known, instead of walking the partials one after another.
 constexpr int kCombineThreads = 256;
 constexpr int kCombineWarps = kCombineThreads / 32;
 
@@ -121,76 +121,56 @@ __global__ void __launch_bounds__(kCombineThreads, 2)
     for (int r = r_lo + warp; r < r_hi; r += kCombineWarps) {
         const size_t orow = static_cast<size_t>(b) * args.R + r;
         const float sink = args.sinks ? args.sinks[r % args.H] : -INFINITY;
-        float4 acc_o[NV4];
-        float lse_all;
-        if (k <= 2) {
-            // two pieces (a sequence cut once, the common case): every lane loads
-            // both lse values and its columns of both partial rows at once (one
-            // round trip)
-            float pl[2];
-            float4 x[2][NV4];
+        auto prow_of = [&](int i) { return static_cast<size_t>(slot_of(i)) * args.R + r; };
+        // the first (up to) 4 partial rows are requested before the lse values
+        // are reduced, so a row cut into at most 4 pieces costs one round trip
+        float4 x[4][NV4];
+        auto load_batch = [&](int i0) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const size_t prow = static_cast<size_t>(slot_of(j)) * args.R + r;
-                pl[j] = args.part_lse[prow];
-                const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
+            for (int j = 0; j < 4; ++j) {
+                if (i0 + j < k) {
+                    const float4* src = reinterpret_cast<const float4*>(args.part_o + prow_of(i0 + j) * DV);
 #pragma unroll
-                for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
-            }
-            const float m = fmaxf(fmaxf(pl[0], pl[1]), sink);
-            const float w0 = expf(pl[0] - m), w1 = expf(pl[1] - m);
-            const float sum = w0 + w1 + expf(sink - m);
-            lse_all = m + logf(sum);
-            const float inv = 1.f / sum;
-#pragma unroll
-            for (int v = 0; v < NV4; ++v) {
-                acc_o[v].x = (w0 * inv) * x[0][v].x + (w1 * inv) * x[1][v].x;
-                acc_o[v].y = (w0 * inv) * x[0][v].y + (w1 * inv) * x[1][v].y;
-                acc_o[v].z = (w0 * inv) * x[0][v].z + (w1 * inv) * x[1][v].z;
-                acc_o[v].w = (w0 * inv) * x[0][v].w + (w1 * inv) * x[1][v].w;
-            }
-        } else {
-            // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
-            float m = -INFINITY;
-            for (int i = lane; i < k; i += 32) m = fmaxf(m, args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            m = fmaxf(m, sink);
-            float sum = 0.f;
-            for (int i = lane; i < k; i += 32) sum += expf(args.part_lse[static_cast<size_t>(slot_of(i)) * args.R + r] - m);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            sum += expf(sink - m);
-            lse_all = m + logf(sum);
-
-            // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
-#pragma unroll
-            for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int i0 = 0; i0 < k; i0 += 4) {
-                float4 x[4][NV4];
-                float w[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int i = i0 + j;
-                    w[j] = 0.f;
-                    if (i < k) {
-                        const size_t prow = static_cast<size_t>(slot_of(i)) * args.R + r;
-                        w[j] = expf(args.part_lse[prow] - lse_all);
-                        const float4* src = reinterpret_cast<const float4*>(args.part_o + prow * DV);
-#pragma unroll
-                        for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
-                    }
+                    for (int v = 0; v < NV4; ++v) x[j][v] = __ldcs(src + lane + 32 * v);
                 }
+            }
+        };
+        load_batch(0);
+        // merged lse: lane i holds piece i (pieces beyond 32 folded in by a loop)
+        const float my_l = lane < k ? args.part_lse[prow_of(lane)] : -INFINITY;
+        float m = my_l;
+        for (int i = lane + 32; i < k; i += 32) m = fmaxf(m, args.part_lse[prow_of(i)]);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (i0 + j < k) {
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        m = fmaxf(m, sink);
+        const float my_e = lane < k ? expf(my_l - m) : 0.f;
+        float sum = my_e;
+        for (int i = lane + 32; i < k; i += 32) sum += expf(args.part_lse[prow_of(i)] - m);
 #pragma unroll
-                        for (int v = 0; v < NV4; ++v) {
-                            acc_o[v].x += w[j] * x[j][v].x;
-                            acc_o[v].y += w[j] * x[j][v].y;
-                            acc_o[v].z += w[j] * x[j][v].z;
-                            acc_o[v].w += w[j] * x[j][v].w;
-                        }
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        sum += expf(sink - m);
+        const float lse_all = m + logf(sum);
+        const float inv = 1.f / sum;
+        const float my_w = my_e * inv;  // weight of piece `lane`: exp(lse_lane - lse)
+
+        // out = sum_i exp(lse_i - lse) * (O_i / l_i); lane owns float4 columns lane + 32 v
+        float4 acc_o[NV4];
+#pragma unroll
+        for (int v = 0; v < NV4; ++v) acc_o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = 0; i0 < k; i0 += 4) {
+            if (i0 > 0) load_batch(i0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = i0 + j;
+                if (i < k) {
+                    const float w = i < 32 ? __shfl_sync(0xffffffffu, my_w, i)
+                                           : expf(args.part_lse[prow_of(i)] - m) * inv;
+#pragma unroll
+                    for (int v = 0; v < NV4; ++v) {
+                        acc_o[v].x += w * x[j][v].x;
+                        acc_o[v].y += w * x[j][v].y;
+                        acc_o[v].z += w * x[j][v].z;
+                        acc_o[v].w += w * x[j][v].w;
                     }
                 }
             }
