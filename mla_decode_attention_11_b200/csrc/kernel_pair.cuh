@@ -94,8 +94,9 @@ struct PairCfg {
 template <int NK, int NV, int NS, int NP>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     mla_decode_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                           const __grid_constant__ CUtensorMap tm_part, const MainArgs args) {
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_pf,
+                           const __grid_constant__ CUtensorMap tm_out, const __grid_constant__ CUtensorMap tm_part,
+                           const MainArgs args) {
     using C = PairCfg<NK, NV, NS, NP>;
     extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -188,6 +189,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
+        ptx::prefetch_tmap(&tm_pf);
         ptx::prefetch_tmap(&tm_out);
         ptx::prefetch_tmap(&tm_part);
     }
@@ -222,17 +224,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     if (warp == 4) {
         // ============================================================ Q + K producer
         if (ptx::elect_one()) {
+            // Each TMA instruction costs the issuing thread a few hundred cycles,
+            // so Q (one box of all 9 chunks) and the prefetches are as large as
+            // the views of q and kv with the chunk index as an outer dimension
+            // allow; K stays one chunk per slot, for a fine-grained ring
             uint32_t k_cnt = 0, piece_cnt = 0;
             int unit = 0;
             bool ok = true;
             // L2 prefetch cursor, `prefetch_tiles` tiles ahead of the K loads
             // through this partition's tiles, across piece boundaries.  A tile
-            // is prefetched whole (all 128 rows, K and V columns alike); on
+            // is prefetched whole (this CTA's 64 rows, K and V columns alike); on
             // entering a later piece the cursor also prefetches that piece's
-            // Q rows, so the Q reload after a piece boundary hits L2.  The two
-            // CTAs split the column chunks.  The cursor starts after the first
-            // piece's Q loads are out and skips the first tile (loaded at once),
-            // so nothing queues ahead of the loads the first MMA needs.
+            // Q rows, so the Q reload after a piece boundary hits L2.  The
+            // cursor starts after the first piece's Q load is out and skips the
+            // first tile (loaded at once), so nothing queues ahead of the loads
+            // the first MMA needs.
             PieceWalker pf_walker = walker;
             Piece pf_pc{};
             bool pf_live = false, pf_started = false;
@@ -241,15 +247,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 if (!pf_live) return;
                 int row0 = pf_t * kTileKV;
                 if (row0 + kTileKV > pf_pc.L) row0 = pf_pc.L - kTileKV;
-                if (issue)
-                    for (int j = static_cast<int>(rank); j < kNumChunks; j += 2)
-                        ptx::tma_prefetch_3d(&tm_v, j * kChunk, row0, pf_pc.b);
+                if (issue) ptx::tma_prefetch_4d(&tm_pf, 0, row0 + static_cast<int>(rank) * 64, 0, pf_pc.b);
                 if (++pf_t == pf_pc.tile_hi) {
                     pf_live = pf_walker.next(pf_pc);
                     if (pf_live) {
                         pf_t = pf_pc.tile_lo;
                         const int qrow = pf_pc.b * args.R + g * 128 + static_cast<int>(rank) * 64;
-                        for (int c = 0; c < kNumChunks; ++c) ptx::tma_prefetch_2d(&tm_q, c * kChunk, qrow);
+                        ptx::tma_prefetch_3d(&tm_q, 0, qrow, 0);
                     }
                 }
             };
@@ -259,9 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 if (!ok) break;
                 if (leader) ptx::mbar_arrive_expect_tx(q_full, 2 * kNumChunks * C::kQChunk);
                 const int qrow = pc.b * args.R + g * 128 + static_cast<int>(rank) * 64;
-                if (!(stall_cta && unit == args.stall_unit))
-                    for (int c = 0; c < kNumChunks; ++c)
-                        ptx::tma_load_2d_pair(q_smem + c * C::kQChunk, &tm_q, lead_q_full, c * kChunk, qrow);
+                if (!(stall_cta && unit == args.stall_unit)) ptx::tma_load_3d_pair(q_smem, &tm_q, lead_q_full, 0, qrow, 0);
                 ++unit;
                 for (int t = pc.tile_lo; t < pc.tile_hi && ok; ++t) {
                     if (!pf_started) {
@@ -323,11 +325,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                         ok = ptx::mbar_wait_bounded(v_empty + s, ((v_cnt / NV) & 1) ^ 1, tmo);
                         if (!ok) break;
                         if (leader) ptx::mbar_arrive_expect_tx(v_full + s, 2 * C::kVSlot);
+                        // this CTA's value columns [col0, col0 + 128): two adjacent chunks, one box
                         const int col0 = 256 * i + 128 * static_cast<int>(rank);
-                        uint8_t* dst = v_smem + s * C::kVSlot;
-                        const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(v_full + s), 0);
-                        ptx::tma_load_3d_pair(dst, &tm_v, bar, col0, row0, pc.b);
-                        ptx::tma_load_3d_pair(dst + C::kVChunk, &tm_v, bar, col0 + 64, row0, pc.b);
+                        ptx::tma_load_4d_pair(v_smem + s * C::kVSlot, &tm_v,
+                                              ptx::mapa_shared(ptx::smem_u32(v_full + s), 0), 0, row0, col0 / kChunk,
+                                              pc.b);
                         ++v_cnt;
                     }
                 }

@@ -126,13 +126,13 @@ constexpr int kDefaultSplitTiles = 16;  // batch-invariant chunks: 16 tiles = 20
 using PairC = mla::PairCfg<kPairNK, kPairNV, kPairNS, kPairNP>;
 
 mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                       const CUtensorMap& tm_v, const CUtensorMap& tm_out, const CUtensorMap& tm_part,
-                       const mla::MainArgs& args, cudaStream_t stream) {
+                       const CUtensorMap& tm_v, const CUtensorMap& tm_pf, const CUtensorMap& tm_out,
+                       const CUtensorMap& tm_part, const mla::MainArgs& args, cudaStream_t stream) {
     auto kern = mla::mla_decode_pair_kernel<kPairNK, kPairNV, kPairNS, kPairNP>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairC::kSmemBytes) != cudaSuccess)
         return MLA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(2 * plan.num_partitions * plan.num_groups));
-    kern<<<grid, PairC::kThreads, PairC::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_out, tm_part, args);
+    kern<<<grid, PairC::kThreads, PairC::kSmemBytes, stream>>>(tm_q, tm_k, tm_v, tm_pf, tm_out, tm_part, args);
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -190,6 +190,35 @@ bool encode_kv(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int
     const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(kv), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// kv viewed with its 64-column chunks as an outer dimension: [B][9 chunks][L_max][64],
+// strides 1152 * L_max, 128, 1152 bytes.  A box of box_rows rows x box_chunks
+// adjacent chunks lands in shared memory chunk after chunk, each chunk a
+// [box_rows][64] block in the same 128-byte swizzle a single-chunk box gives.
+bool encode_kv_chunks(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int B, uint32_t box_rows,
+                      uint32_t box_chunks) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(mla::kChunk), static_cast<cuuint64_t>(L_max),
+                                static_cast<cuuint64_t>(mla::kNumChunks), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(mla::kDqk) * 2, static_cast<cuuint64_t>(mla::kChunk) * 2,
+                                   static_cast<cuuint64_t>(mla::kDqk) * 2 * L_max};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(mla::kChunk), box_rows, box_chunks, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(kv), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// q viewed as [9 chunks][rows][64] (strides 128, 1152 bytes): one box holds
+// 64 rows x all 9 chunks, chunk after chunk
+bool encode_q_chunks(EncodeTiledFn enc, CUtensorMap* m, const void* q, uint64_t rows) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kChunk), rows, static_cast<cuuint64_t>(mla::kNumChunks)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk) * 2, static_cast<cuuint64_t>(mla::kChunk) * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), 64, static_cast<cuuint32_t>(mla::kNumChunks)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -413,14 +442,16 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
     if (!enc) return MLA_ERR_CUDA;
 
     const int G = pl.group_rows;
-    CUtensorMap tm_q, tm_kv, tm_k, tm_out, tm_part;
+    CUtensorMap tm_q, tm_kv, tm_k, tm_pf, tm_out, tm_part;
     if (pl.kernel == MLA_KERNEL_PAIR) {
-        // Q: 64-row halves; K: 64 own kv rows per CTA; V: all 128 rows of a tile;
-        // out and the fp32 partials: the epilogue's TMA stores
+        // Q: 64-row halves, all 9 chunks per box; K: one chunk of 64 own kv rows;
+        // V: 2 chunks x all 128 rows of a tile; L2 prefetch: 64 rows x all 9
+        // chunks; out and the fp32 partials: the epilogue's TMA stores
         uint8_t* part_o = static_cast<uint8_t*>(workspace) + lay.part_o_off;
-        if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, 64) ||
+        if (!encode_q_chunks(enc, &tm_q, q, static_cast<uint64_t>(pl.B) * R) ||
             !encode_kv(enc, &tm_k, kv, pl.L_max, pl.B, 64) ||
-            !encode_kv(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV) ||
+            !encode_kv_chunks(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV, 2) ||
+            !encode_kv_chunks(enc, &tm_pf, kv, pl.L_max, pl.B, 64, mla::kNumChunks) ||
             !encode_rows_store(enc, &tm_out, out, static_cast<uint64_t>(pl.B) * R, false) ||
             !encode_rows_store(enc, &tm_part, part_o, static_cast<uint64_t>(num_slots(pl)) * R, true))
             return MLA_ERR_CUDA;
@@ -470,7 +501,7 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
     if (phases & 1) {
         mla_status st;
         if (pl.kernel == MLA_KERNEL_PAIR)
-            st = launch_pair(pl, tm_q, tm_k, tm_kv, tm_out, tm_part, a, stream);
+            st = launch_pair(pl, tm_q, tm_k, tm_kv, tm_pf, tm_out, tm_part, a, stream);
         else if (pl.kernel == MLA_KERNEL_FP8_MMA)
             st = (G == 16) ? launch_fp8mma<16>(pl, tm_kv, a, stream) : launch_fp8mma<32>(pl, tm_kv, a, stream);
         else if (fp8)
