@@ -407,9 +407,10 @@ def mha_decode_run_phase(plan: mla_plan, q, k, v, seqlens, softmax_scale: float,
 
 def mla_decode_plan_fp8(B: int, Sq: int, H: int, L_max: int, device: Optional[int] = None,
                         num_partitions: int = 0, kernel: int = 0) -> mla_plan:
-    """A plan for a cache of E4M3 codes (mla_decode_plan_fp8): the transposed
-    kernel with FP8 staging, for every head count.  kernel = MLA_KERNEL_FP8_MMA
-    selects the experimental FP8-operand kernel (mla_decode_plan_fp8_kernel)."""
+    """A plan for a cache of E4M3 codes (mla_decode_plan_fp8_kernel).  kernel = 0
+    picks the default, the FP8-operand kernel (MLA_KERNEL_FP8_MMA: the codes as
+    kind::f8f6f4 MMA operands); MLA_KERNEL_FP8 selects the kernel that widens
+    the codes to f16 in shared memory."""
     if device is None:
         device = torch.cuda.current_device()
     p = mla_plan()
