@@ -95,6 +95,18 @@ def test_fp8_empty_and_mixed_lengths(cuda_device, H, kernel):
 
 
 @pytest.mark.parametrize("kernel", FP8_KERNELS)
+def test_fp8_many_short_sequences(cuda_device, kernel):
+    """Far more sequences than partitions, about a tenth of them empty: every
+    partition walks several whole sequences plus cut pieces at its ends."""
+    B, L = 600, 512
+    w = W.custom(B=B, Sq=1, H=128, L=L, seed=760)
+    g = torch.Generator().manual_seed(761)
+    lengths = torch.randint(1, L + 1, (B,), generator=g, dtype=torch.int32)
+    lengths[torch.rand(B, generator=g) < 0.1] = 0
+    check_fp8(w, lengths=lengths, kernel=kernel)
+
+
+@pytest.mark.parametrize("kernel", FP8_KERNELS)
 @pytest.mark.parametrize("H,Sq", [(16, 2), (32, 1), (64, 3), (128, 2)])
 def test_fp8_head_and_token_counts(cuda_device, H, Sq, kernel):
     check_fp8(W.custom(B=2, Sq=Sq, H=H, L=600, seed=160 + H + Sq), kernel=kernel)

@@ -54,6 +54,20 @@ def test_mha_matches_oracle(cuda_device, shape, parts):
     assert_parity(out, lse, ro, rl, f"mha {shape} P={plan.num_partitions}")
 
 
+def test_mha_many_short_sequences(cuda_device):
+    """Far more sequences than partitions (each partition walks several whole
+    sequences plus cut pieces), about a tenth of them empty."""
+    B, L = 500, 384
+    w = W.MhaWorkload("mha_many", B=B, Sq=1, H=32, Hkv=8, L=L, L_lo=1, seed=3100)
+    g = torch.Generator().manual_seed(3101)
+    lengths = torch.randint(1, L + 1, (B,), generator=g, dtype=torch.int32)
+    lengths[torch.rand(B, generator=g) < 0.1] = 0
+    q, k, v, sl = W.generate_mha(w, lengths=lengths)
+    out, lse, plan = run_mha(q, k, v, sl, w.scale)
+    ro, rl = oracle.mha_decode(q, k, v, sl, w.scale)
+    assert_parity(out, lse, ro, rl, f"mha many short P={plan.num_partitions}")
+
+
 def test_mha_sinks(cuda_device):
     w = W.MHA_WORKLOADS["mha_small"]
     q, k, v, sl = W.generate_mha(w)

@@ -110,6 +110,20 @@ def test_empty_and_mixed_lengths(cuda_device, H):
     check_workload(w, lengths=torch.zeros(6, dtype=torch.int32))
 
 
+@pytest.mark.parametrize("B,L,H", [(600, 512, 128), (2000, 256, 16)])
+def test_many_short_sequences(cuda_device, B, L, H):
+    """Far more sequences than partitions, about a tenth of them empty and the
+    rest 1..L keys: every partition walks several whole sequences plus cut
+    pieces at its ends, the length scans take many passes over the batch, and
+    the combine merges the cut ones and writes the empty ones."""
+    w = W.custom(B=B, Sq=1, H=H, L=L, seed=700 + H)
+    g = torch.Generator().manual_seed(701 + H)
+    lengths = torch.randint(1, L + 1, (B,), generator=g, dtype=torch.int32)
+    lengths[torch.rand(B, generator=g) < 0.1] = 0
+    check_workload(w, lengths=lengths)
+    check_workload(w, lengths=lengths, num_partitions=5)
+
+
 @pytest.mark.parametrize("H,Sq", [(16, 1), (16, 2), (16, 3), (32, 1), (64, 1), (128, 1), (128, 2), (64, 3),
                                   (64, 2), (32, 4), (128, 3)])
 def test_head_and_token_counts(cuda_device, H, Sq):
