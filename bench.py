@@ -604,7 +604,8 @@ def run_fp8(args, w: W.Workload):
     torch.cuda.set_device(dev)
     q, codes, ks, sl = W.generate_fp8(w)
     qd, cd, sld = q.to(dev), codes.to(dev), sl.to(dev)
-    kernel = M.MLA_KERNEL_FP8 if args.fp8_kernel == "widen" else M.MLA_KERNEL_FP8_MMA
+    kernel = {"default": 0, "widen": M.MLA_KERNEL_FP8, "operands": M.MLA_KERNEL_FP8_MMA,
+              "pair": M.MLA_KERNEL_FP8_PAIR}[args.fp8_kernel]
     plan = M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=0, kernel=kernel)
     ws = M.alloc_workspace(plan, device=dev)
     M.mla_decode_workspace_init(plan, ws)
@@ -690,25 +691,32 @@ def run_fp8(args, w: W.Workload):
         achieved, peak, unit = nbytes / (main_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
     else:  # f16 MMAs: the measured bf16 figure (same dense rate)
         achieved, peak, unit = flops / (main_ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    traffic, traffic_note = load_traffic(w.name + "_fp8")
+    fp8_kernel_label, fp8_kernel_name, traffic_key = {
+        M.MLA_KERNEL_FP8_PAIR: ("FP8 operands on a CTA pair (kind::f8f6f4)", "mla_decode_pair_fp8_kernel",
+                                w.name + "_fp8"),
+        M.MLA_KERNEL_FP8_MMA: ("FP8 operands (kind::f8f6f4)", "mla_decode_fp8mma_kernel<G>", w.name + "_fp8mma"),
+        M.MLA_KERNEL_FP8: ("transposed (FP8)", "mla_decode_transposed_kernel<G, MlaFp8Shape>", w.name + "_fp8widen"),
+    }[plan.kernel]
+    if plan.kernel == M.MLA_KERNEL_FP8_MMA and plan.kernel == M.mla_decode_plan_fp8(w.B, w.Sq, w.H, w.L, device=-1).kernel:
+        traffic_key = w.name + "_fp8"  # the plan's default kernel for this shape
+    traffic, traffic_note = load_traffic(traffic_key)
     line = {
         "metric": METRIC + " (FP8 latent cache)",
         "value": flops / (t_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e4m3 cache, e4m3 MMA" if kernel == M.MLA_KERNEL_FP8_MMA else "e4m3 cache, f16 MMA",
+        "dtype": "e4m3 cache, f16 MMA" if plan.kernel == M.MLA_KERNEL_FP8 else "e4m3 cache, e4m3 MMA",
         "data": "synthetic",
         "config": {"workload": workload_desc(w) + f"; cache quantised to E4M3, kv_scale = amax/448 = {ks:.6g}",
                    "global_batch": w.B, "seq_len": w.L, "parallelism": "single GPU",
-                   "kernel": "FP8 operands (kind::f8f6f4)" if kernel == M.MLA_KERNEL_FP8_MMA else "transposed (FP8)",
+                   "kernel": fp8_kernel_label,
                    "group_rows": plan.group_rows, "partitions": plan.num_partitions,
                    "l2": l2_note(codes.numel())},
         "hbm_gbs": nbytes / (t_ms * 1e-3) / 1e9,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                      "traffic_note": traffic_note,
-                     "kernel": ("mla_decode_fp8mma_kernel<G>" if kernel == M.MLA_KERNEL_FP8_MMA
-                                else "mla_decode_transposed_kernel<G, MlaFp8Shape>"), "kernel_ms": main_ms,
+                     "kernel": fp8_kernel_name, "kernel_ms": main_ms,
                      "combine_ms": comb_ms, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
                      "hbm_frac": nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "step_roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
@@ -737,8 +745,9 @@ def main():
                     help="time the attention-sink entry point (per-head sink logits) on the same workload")
     ap.add_argument("--fp8", action="store_true",
                     help="the same MLA workload over an FP8 (E4M3) latent cache (mla_decode_run_fp8)")
-    ap.add_argument("--fp8-kernel", choices=["operands", "widen"], default="operands",
-                    help="FP8 cache kernel: codes as kind::f8f6f4 MMA operands (default) or widened to f16")
+    ap.add_argument("--fp8-kernel", choices=["default", "pair", "operands", "widen"], default="default",
+                    help="FP8 cache kernel: the plan's default, the CTA-pair operand kernel (Sq*H % 128 == 0), "
+                         "the transposed operand kernel, or the widening kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

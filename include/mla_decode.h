@@ -65,8 +65,10 @@ enum {
     MLA_KERNEL_MHA = 3,        /* MHA decode (mha_decode_plan): the transposed kernel over 128-wide K, V */
     MLA_KERNEL_FP8 = 4,        /* MLA decode over an FP8 cache (mla_decode_plan_fp8): the transposed kernel
                                   with E4M3 chunks widened to f16 in shared memory */
-    MLA_KERNEL_FP8_MMA = 5     /* MLA decode over an FP8 cache with the codes as kind::f8f6f4 MMA operands
+    MLA_KERNEL_FP8_MMA = 5,    /* MLA decode over an FP8 cache with the codes as kind::f8f6f4 MMA operands
                                   (what mla_decode_plan_fp8 picks; see mla_decode_plan_fp8_kernel) */
+    MLA_KERNEL_FP8_PAIR = 6    /* MLA decode over an FP8 cache on a CTA pair: the pair kernel's dataflow with
+                                  the codes as kind::f8f6f4 operands (H*Sq % 128 == 0) */
 };
 
 /*
@@ -339,8 +341,14 @@ mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void*
  * at the top of this file on those values (keys: all 576 columns; values:
  * the first 512), with q bf16, out bf16 and lse fp32 as there.
  *
- * Numerics, by kernel (both keep the cache's values exact and accumulate in fp32):
- *   MLA_KERNEL_FP8_MMA (the default): the codes are the operands of
+ * Numerics, by kernel (all keep the cache's values exact and accumulate in fp32):
+ *   MLA_KERNEL_FP8_PAIR (the default when Sq*H is a multiple of 128): the
+ *     codes are the operands of kind::f8f6f4 MMAs on a CTA pair; each q row is
+ *     scaled by a power of two and carried as the sum of two E4M3 terms (about
+ *     8 significant bits, the precision of a bf16 q), and P (scaled by 2^7) as
+ *     the sum of two (about 8 bits, the precision of the bf16 P of the bf16
+ *     path).
+ *   MLA_KERNEL_FP8_MMA (the default otherwise): the codes are the operands of
  *     kind::f8f6f4 tensor-core MMAs as they are; each q row is scaled by a
  *     power of two and carried as the sum of three E4M3 terms (about 12
  *     significant bits, relative error <= 2^-12), and P (scaled by 2^7) as the
@@ -353,16 +361,21 @@ mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void*
  *     the scores (with softmax_scale) and the output rows.
  *
  * mla_decode_plan_fp8 -- as mla_decode_plan (same arguments, limits and return
- * codes) for an FP8 cache; the plan's kernel is MLA_KERNEL_FP8_MMA (16 or 32
- * query rows per CTA, 192 threads), for every head count.
+ * codes) for an FP8 cache; the plan's kernel is MLA_KERNEL_FP8_PAIR (128-row
+ * query groups on CTA pairs, 256 threads, the bf16 pair plan's partitions) when
+ * Sq*H is a multiple of 128, else MLA_KERNEL_FP8_MMA (16 or 32 query rows per
+ * CTA, 192 threads).
  */
 mla_status mla_decode_plan_fp8(int32_t B, int32_t Sq, int32_t H, int32_t L_max, int32_t device,
                                int32_t num_partitions_override, mla_plan* plan, size_t* workspace_bytes);
 
 /*
  * mla_decode_plan_fp8_kernel -- mla_decode_plan_fp8 with an explicit kernel:
- *   kernel  0 or MLA_KERNEL_FP8_MMA: the codes as MMA operands (what
- *           mla_decode_plan_fp8 picks; q and P carried as sums of E4M3 terms);
+ *   kernel  0: what mla_decode_plan_fp8 picks;
+ *           MLA_KERNEL_FP8_PAIR: the codes as MMA operands on CTA pairs
+ *           (MLA_ERR_UNSUPPORTED unless Sq*H % 128 == 0);
+ *           MLA_KERNEL_FP8_MMA: the codes as MMA operands, transposed
+ *           orientation, any supported shape;
  *           MLA_KERNEL_FP8: the widening kernel (f16 operands, 320 threads).
  *           Anything else: MLA_ERR_INVALID_ARG.
  * Other arguments and return codes as mla_decode_plan_fp8; the plan runs

@@ -35,6 +35,7 @@ MLA_KERNEL_PAIR = 2
 MLA_KERNEL_MHA = 3
 MLA_KERNEL_FP8 = 4
 MLA_KERNEL_FP8_MMA = 5
+MLA_KERNEL_FP8_PAIR = 6
 MHA_D = 128
 MLA_NOALLOC_SCRATCH_BYTES = 40 * 1024 * 1024
 
@@ -408,9 +409,10 @@ def mha_decode_run_phase(plan: mla_plan, q, k, v, seqlens, softmax_scale: float,
 def mla_decode_plan_fp8(B: int, Sq: int, H: int, L_max: int, device: Optional[int] = None,
                         num_partitions: int = 0, kernel: int = 0) -> mla_plan:
     """A plan for a cache of E4M3 codes (mla_decode_plan_fp8_kernel).  kernel = 0
-    picks the default, the FP8-operand kernel (MLA_KERNEL_FP8_MMA: the codes as
-    kind::f8f6f4 MMA operands); MLA_KERNEL_FP8 selects the kernel that widens
-    the codes to f16 in shared memory."""
+    picks the default: the codes as kind::f8f6f4 MMA operands on CTA pairs
+    (MLA_KERNEL_FP8_PAIR) when Sq*H is a multiple of 128, else in the
+    transposed orientation (MLA_KERNEL_FP8_MMA); MLA_KERNEL_FP8 selects the
+    kernel that widens the codes to f16 in shared memory."""
     if device is None:
         device = torch.cuda.current_device()
     p = mla_plan()

@@ -18,6 +18,7 @@
 
 #include "../../include/mla_decode.h"
 #include "kernel_combine.cuh"
+#include "kernel_pair_fp8.cuh"
 #include "kernel_pair.cuh"
 #include "kernel_transposed.cuh"
 #include "kernel_fp8mma.cuh"
@@ -136,6 +137,21 @@ mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUte
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+constexpr int kPairFp8NK = 14;  // K chunks of 4 KB
+constexpr int kPairFp8NV = 4;   // V slots of 16 KB (two tiles)
+using PairFp8C = mla::PairFp8Cfg<kPairFp8NK, kPairFp8NV, kPairNS, kPairNP>;
+
+mla_status launch_pair_fp8(const mla_plan& plan, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                           const CUtensorMap& tm_pf, const CUtensorMap& tm_out, const CUtensorMap& tm_part,
+                           const mla::MainArgs& args, cudaStream_t stream) {
+    auto kern = mla::mla_decode_pair_fp8_kernel<kPairFp8NK, kPairFp8NV, kPairNS, kPairNP>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairFp8C::kSmemBytes) != cudaSuccess)
+        return MLA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(2 * plan.num_partitions * plan.num_groups));
+    kern<<<grid, PairFp8C::kThreads, PairFp8C::kSmemBytes, stream>>>(tm_k, tm_v, tm_pf, tm_out, tm_part, args);
+    return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
 // Output maps of the pair kernel's TMA-store epilogue: rows of 512 values,
 // boxes of 32 rows x 128 bytes (64 bf16 or 32 fp32 columns), 128-byte swizzle.
 bool encode_rows_store(EncodeTiledFn enc, CUtensorMap* m, const void* base, uint64_t rows, bool fp32) {
@@ -223,16 +239,33 @@ bool encode_q_chunks(EncodeTiledFn enc, CUtensorMap* m, const void* q, uint64_t 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// FP8 cache: kv viewed as [B][L_max][576] bytes (E4M3 codes): a box of 128
-// rows x 64 codes, 64-byte swizzle (rows of 64 bytes)
-bool encode_kv_fp8(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int B) {
+// FP8 cache: kv viewed as [B][L_max][576] bytes (E4M3 codes): a box of
+// box_rows rows x 64 codes, 64-byte swizzle (rows of 64 bytes)
+bool encode_kv_fp8(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int B, uint32_t box_rows) {
     const cuuint64_t dims[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(L_max),
                                 static_cast<cuuint64_t>(B)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(mla::kDqk),
                                    static_cast<cuuint64_t>(mla::kDqk) * L_max};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), static_cast<cuuint32_t>(mla::kTileKV), 1};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(mla::kChunk), box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(kv), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// FP8 cache with its 64-code chunks as an outer dimension: [B][9 chunks][L_max][64]
+// bytes, strides 576 * L_max, 64, 576.  A box of box_rows rows x box_chunks
+// adjacent chunks lands chunk after chunk, each a [box_rows][64] block in the
+// 64-byte swizzle a single-chunk box gives.
+bool encode_kv_fp8_chunks(EncodeTiledFn enc, CUtensorMap* m, const void* kv, int L_max, int B, uint32_t box_rows,
+                          uint32_t box_chunks) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(mla::kChunk), static_cast<cuuint64_t>(L_max),
+                                static_cast<cuuint64_t>(mla::kNumChunks), static_cast<cuuint64_t>(B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(mla::kDqk), static_cast<cuuint64_t>(mla::kChunk),
+                                   static_cast<cuuint64_t>(mla::kDqk) * L_max};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(mla::kChunk), box_rows, box_chunks, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(kv), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -343,14 +376,25 @@ mla_status mla_decode_plan_fp8_kernel(int32_t B, int32_t Sq, int32_t H, int32_t 
                                       int32_t num_partitions_override, int32_t kernel, mla_plan* plan,
                                       size_t* workspace_bytes) {
     if (!plan) return MLA_ERR_INVALID_ARG;
-    // default: the codes as kind::f8f6f4 operands (2.3x the widening kernel on a B200)
-    if (kernel == 0) kernel = MLA_KERNEL_FP8_MMA;
-    if (kernel != MLA_KERNEL_FP8 && kernel != MLA_KERNEL_FP8_MMA) return MLA_ERR_INVALID_ARG;
+    // default: the codes as kind::f8f6f4 operands; on a CTA pair when Sq * H is a
+    // multiple of 128 (1.4x the transposed operand kernel there), else the
+    // transposed operand kernel (2.3x the widening kernel on a B200)
+    if (kernel == 0) kernel = ((Sq * H) % 128 == 0) ? MLA_KERNEL_FP8_PAIR : MLA_KERNEL_FP8_MMA;
+    if (kernel != MLA_KERNEL_FP8 && kernel != MLA_KERNEL_FP8_MMA && kernel != MLA_KERNEL_FP8_PAIR)
+        return MLA_ERR_INVALID_ARG;
     mla_plan p;
-    const mla_status st =
-        mla_decode_plan_kernel(B, Sq, H, L_max, device, num_partitions_override, MLA_KERNEL_TRANSPOSED, &p, nullptr);
+    const mla_status st = mla_decode_plan_kernel(B, Sq, H, L_max, device, num_partitions_override,
+                                                 kernel == MLA_KERNEL_FP8_PAIR ? MLA_KERNEL_PAIR : MLA_KERNEL_TRANSPOSED,
+                                                 &p, nullptr);
     if (st != MLA_OK) return st;
     p.kernel = kernel;
+    if (kernel == MLA_KERNEL_FP8_PAIR) {  // the pair plan's groups and partitions
+        p.cta_threads = PairFp8C::kThreads;
+        p.smem_bytes = PairFp8C::kSmemBytes;
+        *plan = p;
+        if (workspace_bytes) *workspace_bytes = p.workspace_bytes;
+        return MLA_OK;
+    }
     const bool g16 = (p.group_rows == 16);
     if (kernel == MLA_KERNEL_FP8) {
         p.cta_threads = g16 ? mla::TransposedCfg<16, mla::MlaFp8Shape>::kThreads
@@ -389,7 +433,8 @@ mla_status check_run_args(const mla_plan* plan, const void* q, const void* kv, c
     if (phases < 1 || phases > 3) return MLA_ERR_INVALID_ARG;
     if (!plan || !q || !kv || !seqlens || !out || !lse) return MLA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale)) return MLA_ERR_INVALID_ARG;
-    const bool fp8 = (plan->kernel == MLA_KERNEL_FP8 || plan->kernel == MLA_KERNEL_FP8_MMA);
+    const bool fp8 = (plan->kernel == MLA_KERNEL_FP8 || plan->kernel == MLA_KERNEL_FP8_MMA ||
+                      plan->kernel == MLA_KERNEL_FP8_PAIR);
     if (fp8 != (kv_scale != nullptr)) return MLA_ERR_INVALID_ARG;  // plan kind and entry point disagree
     if (fp8 && !(std::isfinite(*kv_scale) && *kv_scale > 0.f)) return MLA_ERR_INVALID_ARG;
     const mla_plan& pl = *plan;
@@ -399,9 +444,9 @@ mla_status check_run_args(const mla_plan* plan, const void* q, const void* kv, c
         return MLA_ERR_INVALID_ARG;
     if (pl.l2_prefetch_tiles < 0 || pl.l2_prefetch_tiles > 16) return MLA_ERR_INVALID_ARG;
     if (pl.split_tiles < 0 || pl.split_tiles > (1 << 17)) return MLA_ERR_INVALID_ARG;
-    if (pl.kernel == MLA_KERNEL_TRANSPOSED || fp8) {
+    if (pl.kernel == MLA_KERNEL_TRANSPOSED || pl.kernel == MLA_KERNEL_FP8 || pl.kernel == MLA_KERNEL_FP8_MMA) {
         if (pl.group_rows != 16 && pl.group_rows != 32) return MLA_ERR_INVALID_ARG;
-    } else if (pl.kernel == MLA_KERNEL_PAIR) {
+    } else if (pl.kernel == MLA_KERNEL_PAIR || pl.kernel == MLA_KERNEL_FP8_PAIR) {
         if (pl.group_rows != 128) return MLA_ERR_INVALID_ARG;
     } else {
         return MLA_ERR_INVALID_ARG;  // MHA plans run through mha_decode_run
@@ -435,7 +480,7 @@ mla_status check_run_device(const mla_plan& pl) {
 mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, const int32_t* seqlens,
                          float softmax_scale, const float* sinks, void* out, float* lse, void* workspace,
                          void* stream_, int phases, const float* kv_scale) {
-    const bool fp8 = (pl.kernel == MLA_KERNEL_FP8 || pl.kernel == MLA_KERNEL_FP8_MMA);
+    const bool fp8 = (pl.kernel == MLA_KERNEL_FP8 || pl.kernel == MLA_KERNEL_FP8_MMA || pl.kernel == MLA_KERNEL_FP8_PAIR);
     const int R = pl.Sq * pl.H;
     const Layout lay = workspace_layout(num_slots(pl), R);
     EncodeTiledFn enc = encode_fn();
@@ -455,9 +500,20 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
             !encode_rows_store(enc, &tm_out, out, static_cast<uint64_t>(pl.B) * R, false) ||
             !encode_rows_store(enc, &tm_part, part_o, static_cast<uint64_t>(num_slots(pl)) * R, true))
             return MLA_ERR_CUDA;
+    } else if (pl.kernel == MLA_KERNEL_FP8_PAIR) {
+        // K: one 64-code chunk of 64 own kv rows; V: 2 chunks x all 128 rows of a
+        // tile; L2 prefetch: 64 rows x all 9 chunks (64-byte swizzle); Q terms are
+        // written by the kernel from q; out and the fp32 partials as for bf16
+        uint8_t* part_o = static_cast<uint8_t*>(workspace) + lay.part_o_off;
+        if (!encode_kv_fp8(enc, &tm_k, kv, pl.L_max, pl.B, 64) ||
+            !encode_kv_fp8_chunks(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV, 2) ||
+            !encode_kv_fp8_chunks(enc, &tm_pf, kv, pl.L_max, pl.B, 64, mla::kNumChunks) ||
+            !encode_rows_store(enc, &tm_out, out, static_cast<uint64_t>(pl.B) * R, false) ||
+            !encode_rows_store(enc, &tm_part, part_o, static_cast<uint64_t>(num_slots(pl)) * R, true))
+            return MLA_ERR_CUDA;
     } else if (fp8) {
         if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, G) ||
-            !encode_kv_fp8(enc, &tm_kv, kv, pl.L_max, pl.B))
+            !encode_kv_fp8(enc, &tm_kv, kv, pl.L_max, pl.B, mla::kTileKV))
             return MLA_ERR_CUDA;
     } else {
         if (!encode_2d_bf16(enc, &tm_q, q, mla::kDqk, static_cast<uint64_t>(pl.B) * R, mla::kChunk, G) ||
@@ -502,6 +558,8 @@ mla_status launch_phases(const mla_plan& pl, const void* q, const void* kv, cons
         mla_status st;
         if (pl.kernel == MLA_KERNEL_PAIR)
             st = launch_pair(pl, tm_q, tm_k, tm_kv, tm_pf, tm_out, tm_part, a, stream);
+        else if (pl.kernel == MLA_KERNEL_FP8_PAIR)
+            st = launch_pair_fp8(pl, tm_k, tm_kv, tm_pf, tm_out, tm_part, a, stream);
         else if (pl.kernel == MLA_KERNEL_FP8_MMA)
             st = (G == 16) ? launch_fp8mma<16>(pl, tm_kv, a, stream) : launch_fp8mma<32>(pl, tm_kv, a, stream);
         else if (fp8)

@@ -165,15 +165,26 @@ def test_fp8_run_rejects_without_launching(lib):
 
 
 def test_fp8_operand_kernel_plan_without_gpu():
-    """The FP8-operand kernel is the default FP8 plan; the widening kernel is
-    chosen explicitly; other kinds are refused."""
+    """The FP8 operand kernels are the default FP8 plans: on a CTA pair when
+    Sq*H is a multiple of 128, else the transposed one; the others are chosen
+    explicitly; other kinds are refused, the pair kernel for shapes it cannot run."""
     for H, G in ((16, 16), (128, 32)):
-        p = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1)
-        assert p.kernel == M.MLA_KERNEL_FP8_MMA and p.group_rows == G and p.cta_threads == 192
-        assert p.smem_bytes <= 232448
+        o = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8_MMA)
+        assert o.kernel == M.MLA_KERNEL_FP8_MMA and o.group_rows == G and o.cta_threads == 192
+        assert o.smem_bytes <= 232448
         w = M.mla_decode_plan_fp8(8, 1, H, 4096, device=-1, kernel=M.MLA_KERNEL_FP8)
         assert w.kernel == M.MLA_KERNEL_FP8 and w.group_rows == G
-    for bad in (1, 2, 3, 6):
+    assert M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1).kernel == M.MLA_KERNEL_FP8_MMA
+    for Sq, H in ((1, 128), (2, 64), (2, 128)):
+        p = M.mla_decode_plan_fp8(8, Sq, H, 4096, device=-1)
+        bf = M.mla_decode_plan(8, Sq, H, 4096, device=-1)
+        assert p.kernel == M.MLA_KERNEL_FP8_PAIR and p.group_rows == 128 and p.cta_threads == 256
+        assert p.num_groups == bf.num_groups and p.num_partitions == bf.num_partitions
+        assert p.workspace_bytes == bf.workspace_bytes and p.smem_bytes <= 232448
+    with pytest.raises(M.MlaError) as e:
+        M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1, kernel=M.MLA_KERNEL_FP8_PAIR)
+    assert e.value.code == 3
+    for bad in (1, 2, 3, 7):
         with pytest.raises(M.MlaError) as e:
             M.mla_decode_plan_fp8(8, 1, 16, 4096, device=-1, kernel=bad)
         assert e.value.code == 1

@@ -1,14 +1,16 @@
 """GPU parity of the FP8-cache entry point (mla_decode_plan_fp8 /
 mla_decode_run_fp8) against the fp64 oracle's FP8 definition: E4M3 codes,
-value = kv_scale * e4m3(code), q bf16.  Both FP8 kernels (the codes as
-kind::f8f6f4 MMA operands, the default, and the widening kernel), both group
-sizes (16 and 32 query rows per CTA), unsplit and split sequences, lengths
+value = kv_scale * e4m3(code), q bf16.  The three FP8 kernels (the codes as
+kind::f8f6f4 MMA operands on a CTA pair and in the transposed orientation, the
+defaults, and the widening kernel), every group size (16, 32 and 128 query
+rows), unsplit and split sequences, lengths
 around tile edges, empty sequences, sinks, every finite code, full sizes on
 sampled rows.  Rows past a length hold the NaN code (NaN to the oracle,
 +-480 * kv_scale to the widening kernel, NaN to the operand kernel; both require
 finite codes), so a read past a length would break parity.  Tolerances as in test_gpu_parity (the
 cache values are exact in both kernels; q carries about 12 significant bits in
-the operand kernel and P about 8, the precision of the bf16 path's P)."""
+the transposed operand kernel, about 8 in the pair kernel, and P about 8, the
+precision of the bf16 path's P)."""
 import math
 
 import numpy as np
@@ -25,11 +27,15 @@ pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
 
 
-# the FP8 kernels these tests cover: the codes as MMA operands (default) and the widening kernel
-FP8_KERNELS = [M.MLA_KERNEL_FP8_MMA, M.MLA_KERNEL_FP8]
+# the FP8 kernels these tests cover: the codes as MMA operands on a CTA pair (the
+# default when Sq*H % 128 == 0) and in the transposed orientation (the default
+# otherwise), and the widening kernel
+FP8_KERNELS = [M.MLA_KERNEL_FP8_PAIR, M.MLA_KERNEL_FP8_MMA, M.MLA_KERNEL_FP8]
 
 
 def gpu_decode_fp8(q, codes, ks, sl, scale, num_partitions=0, sinks=None, kernel=M.MLA_KERNEL_FP8_MMA):
+    if kernel == M.MLA_KERNEL_FP8_PAIR and (q.shape[1] * q.shape[2]) % 128 != 0:
+        pytest.skip("the CTA-pair FP8 kernel runs 128-row query groups (Sq*H % 128 == 0)")
     plan = M.mla_decode_plan_fp8(q.shape[0], q.shape[1], q.shape[2], codes.shape[1], device=0,
                                  num_partitions=num_partitions, kernel=kernel)
     assert plan.kernel == kernel
@@ -67,7 +73,10 @@ SMALL = {
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_fp8_small_workloads(cuda_device, name, kernel):
     _, plan = check_fp8(SMALL[name], kernel=kernel)
-    assert plan.group_rows == (16 if SMALL[name].Sq * SMALL[name].H == 16 else 32)
+    if kernel == M.MLA_KERNEL_FP8_PAIR:
+        assert plan.group_rows == 128
+    else:
+        assert plan.group_rows == (16 if SMALL[name].Sq * SMALL[name].H == 16 else 32)
 
 
 @pytest.mark.parametrize("kernel", FP8_KERNELS)
@@ -80,6 +89,9 @@ def test_fp8_forced_partitions(cuda_device, parts, H, kernel):
 @pytest.mark.parametrize("kernel", FP8_KERNELS)
 @pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 127, 128, 129, 255, 257, 1023])
 def test_fp8_lengths_around_tile_edges(cuda_device, L, kernel):
+    if kernel == M.MLA_KERNEL_FP8_PAIR:
+        check_fp8(W.custom(B=2, Sq=1, H=128, L=L, seed=142 + L), kernel=kernel)
+        return
     check_fp8(W.custom(B=2, Sq=1, H=16, L=L, seed=140 + L), kernel=kernel)
     check_fp8(W.custom(B=1, Sq=1, H=64, L=L, seed=141 + L), kernel=kernel)
 
@@ -130,6 +142,8 @@ def test_fp8_every_finite_code(cuda_device, kernel):
     scale, so the max-abs bound is scaled by max(1, max|ref|) as in the
     large-score test of test_gpu_parity."""
     for H, seed in ((16, 180), (128, 181)):
+        if kernel == M.MLA_KERNEL_FP8_PAIR and H != 128:
+            continue
         g = torch.Generator().manual_seed(seed)
         B, L = 2, 700
         codes = torch.randint(0, 256, (B, L, 576), generator=g, dtype=torch.int64).to(torch.uint8)
@@ -148,7 +162,7 @@ def test_fp8_every_finite_code(cuda_device, kernel):
 def test_fp8_large_scale_and_rescale(cuda_device, kernel):
     """A kv_scale that makes the scaled scores span tens of units: the lazy
     online rescale runs on the FP8 path too."""
-    w = W.custom(B=2, Sq=1, H=16, L=2000, sigma=3.0, seed=190)
+    w = W.custom(B=2, Sq=1, H=128 if kernel == M.MLA_KERNEL_FP8_PAIR else 16, L=2000, sigma=3.0, seed=190)
     q, codes, ks, sl = W.generate_fp8(w)
     out, lse, _ = gpu_decode_fp8(q, codes, ks, sl, w.scale, kernel=kernel)
     ro, rl = oracle.mla_decode_fp8(q, codes, ks, sl, w.scale)
@@ -165,7 +179,7 @@ def test_fp8_deterministic_and_split_invariant(cuda_device, kernel):
     assert torch.equal(l1, l2)
     o3, l3, _ = gpu_decode_fp8(q, codes, ks, sl, w.scale, num_partitions=1, kernel=kernel)
     assert (o1.double() - o3.double()).abs().max().item() <= 1e-2
-    # The operand kernel carries P as two E4M3 terms (about 8 significant bits)
+    # The operand kernels carry P as two E4M3 terms (about 8 significant bits)
     # rounded against the running reference max, which moves at other points
     # when a sequence is cut: its lse may differ between splits by the rounding
     # of P (measured 1.8e-4), bounded here by the lse parity tolerance.  The
@@ -201,6 +215,8 @@ def test_fp8_bounded_wait_timeout_reports_and_recovers(cuda_device, H, kernel):
     """Host-side fault injection as in test_gpu_parity: the producer of CTA 0
     skips one load it armed; the bounded waits (converters and MMA issuer)
     run out, MLA_ERR_TIMEOUT is reported, and the next run is clean."""
+    if kernel == M.MLA_KERNEL_FP8_PAIR and H % 128 != 0:
+        pytest.skip("the CTA-pair FP8 kernel runs 128-row query groups (Sq*H % 128 == 0)")
     w = W.custom(B=2, Sq=1, H=H, L=1000, seed=201)
     q, codes, ks, sl = W.generate_fp8(w)
     plan = M.mla_decode_plan_fp8(2, 1, H, 1000, device=0, kernel=kernel)
