@@ -13,9 +13,10 @@
 //      about 8 significant bits (the precision of a bf16 q).  Both terms
 //      multiply the same K chunk into the same S accumulator, so
 //      S = (t1 + t2) K^T and the softmax multiplies each row by 2^-e.
-//   P: carried as 2^7 p and written as two E4M3 terms (about 8 significant
-//      bits, the precision of the bf16 P of the other kernels); both multiply
-//      the same V chunk into O.  The row sum adds the same two terms, so the
+//   P: carried as 2^7 p, rounded to f16 and written as two E4M3 terms
+//      t1 = e4m3(h), t2 = e4m3(h - t1) (about 8 significant bits, the
+//      precision of the bf16 P of the other kernels); both multiply the same
+//      V chunk into O.  The row sum adds the fp32 weights 2^7 p, so the
 //      factor 2^7 cancels in O / l; the reference max is raised whenever a row
 //      max exceeds it by more than 1 (base 2), so 2^7 p <= 256 stays inside
 //      E4M3 while small weights keep normal codes.
@@ -29,6 +30,8 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cstdint>
 
 #include "kernel_fp8mma.cuh"
@@ -37,6 +40,19 @@
 #include "schedule.cuh"
 
 namespace mla {
+
+// An f16 pair -> two E4M3 codes (round to nearest even, saturating at +-448);
+// the low byte holds the low half.
+__device__ __forceinline__ uint32_t f16x2_to_e4m3x2(__half2 h) {
+    return static_cast<uint32_t>(
+        __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&h), __NV_SATFINITE, __NV_E4M3));
+}
+
+// The two values of an E4M3 code pair as an f16 pair, exactly.
+__device__ __forceinline__ __half2 e4m3x2_to_f16x2(uint32_t codes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(codes & 0xFFFFu), __NV_E4M3);
+    return *reinterpret_cast<const __half2*>(&h);
+}
 
 template <int NK, int NV, int NS, int NP>
 struct PairFp8Cfg {
@@ -620,23 +636,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                         float a[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) a[i] = ex2_approx(fmaf(x[4 * e + i], cs, -mm));
-                        // first term: a rounded to 4 significant bits (round half away
-                        // from zero on the float bits), which E4M3 holds exactly for
-                        // a in [2^-6, 448]; second term: the remainder, rounded by the
-                        // conversion.  (Below 2^-6 the first term rounds once more, to
-                        // E4M3's subnormal spacing 2^-9: an error under 2^-16 of the row
-                        // sum, whose largest term is 2^7.)  The row sum takes the fp32
-                        // weights, as in the bf16 kernel.
-                        float v[4], rem[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            v[i] = __uint_as_float((__float_as_uint(a[i]) + 0x80000u) & 0xFFF00000u);
-                            rem[i] = a[i] - v[i];
-                        }
-                        const uint32_t c01 = f32x2_to_e4m3x2(v[0], v[1]);
-                        const uint32_t c23 = f32x2_to_e4m3x2(v[2], v[3]);
-                        const uint32_t d01 = f32x2_to_e4m3x2(rem[0], rem[1]);
-                        const uint32_t d23 = f32x2_to_e4m3x2(rem[2], rem[3]);
+                        // Two terms through f16 pairs: h = a rounded to f16 (relative
+                        // error 2^-11); first term = h rounded to E4M3; the remainder
+                        // h - first is exact in f16 (a multiple of h's spacing, at most
+                        // half the first term's spacing, so under 8 significant bits);
+                        // second term = the remainder rounded to E4M3.  The pair holds a
+                        // to about 2^-8 relative (below E4M3's normal range, to its
+                        // subnormal spacing 2^-9: under 2^-16 of the row sum, whose
+                        // largest term is 2^7).  The row sum takes the fp32 weights, as
+                        // in the bf16 kernel.
+                        const __half2 h01 = __floats2half2_rn(a[0], a[1]);
+                        const __half2 h23 = __floats2half2_rn(a[2], a[3]);
+                        const uint32_t c01 = f16x2_to_e4m3x2(h01);
+                        const uint32_t c23 = f16x2_to_e4m3x2(h23);
+                        const uint32_t d01 = f16x2_to_e4m3x2(__hsub2(h01, e4m3x2_to_f16x2(c01)));
+                        const uint32_t d23 = f16x2_to_e4m3x2(__hsub2(h23, e4m3x2_to_f16x2(c23)));
                         lsum += (a[0] + a[1]) + (a[2] + a[3]);
                         packed[0][e] = c01 | (c23 << 16);
                         packed[1][e] = d01 | (d23 << 16);
