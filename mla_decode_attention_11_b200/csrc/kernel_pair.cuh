@@ -523,16 +523,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                     for (int j = 0; j < 64; ++j)
                         if (kv0 + j < lo) x[j] = -INFINITY;
                 }
-                // this thread's max (pairwise tree), then published for the row's
-                // other thread; the exchange completes while the exps below run
-                float mt[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) mt[j] = fmaxf(x[2 * j], x[2 * j + 1]);
-#pragma unroll
-                for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                    for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
-                const float mloc = mt[0] * cs;
+                // this thread's max (a tree of three-input maxima), then published
+                // for the row's other thread; the exchange completes while the
+                // exps below run
+                const float mloc = ptx::max64(x) * cs;
                 float* redmax = red + (tile_cnt & 1) * 128;
                 redmax[L_id] = mloc;
                 ptx::mbar_arrive(group_sync);
@@ -543,15 +537,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 uint32_t packed[32];
                 float lsum = 0.f;
                 auto exps = [&](float m) {
-                    lsum = 0.f;
+                    // the exponents and the row sum two lanes at a time (packed fp32)
+                    float2 ls = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const float a0 = ex2_approx(fmaf(x[2 * e], cs, -m));
-                        const float a1 = ex2_approx(fmaf(x[2 * e + 1], cs, -m));
-                        lsum += a0 + a1;
+                        const float2 tt = ptx::ffma2(make_float2(x[2 * e], x[2 * e + 1]), make_float2(cs, cs),
+                                                     make_float2(-m, -m));
+                        const float a0 = ex2_approx(tt.x);
+                        const float a1 = ex2_approx(tt.y);
+                        ls = ptx::fadd2(ls, make_float2(a0, a1));
                         const __nv_bfloat162 hv = __floats2bfloat162_rn(a0, a1);
                         packed[e] = *reinterpret_cast<const uint32_t*>(&hv);
                     }
+                    lsum = ls.x + ls.y;
                 };
                 if (!first) exps(m_ref);
                 ok = ptx::mbar_wait_bounded(group_sync, sync_cnt & 1, tmo);

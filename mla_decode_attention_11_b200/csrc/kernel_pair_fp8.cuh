@@ -608,16 +608,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                     for (int j = 0; j < 64; ++j)
                         if (kv0 + j < lo) x[j] = -INFINITY;
                 }
-                // this thread's max (pairwise tree), then published for the row's
-                // other thread; the exchange completes while the exps below run
-                float mt[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) mt[j] = fmaxf(x[2 * j], x[2 * j + 1]);
-#pragma unroll
-                for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-                    for (int j = 0; j < w; ++j) mt[j] = fmaxf(mt[j], mt[j + w]);
-                const float mloc = mt[0] * cs;
+                // this thread's max (a tree of three-input maxima), then published
+                // for the row's other thread; the exchange completes while the
+                // exps below run
+                const float mloc = ptx::max64(x) * cs;
                 float* redmax = red + (tile_cnt & 1) * 128;
                 redmax[L_id] = mloc;
                 ptx::mbar_arrive(group_sync);
@@ -629,13 +623,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 uint32_t packed[2][16];  // term k: 64 codes in 16 words
                 float lsum = 0.f;
                 auto exps = [&](float m) {
-                    lsum = 0.f;
+                    // the exponents and the row sum two lanes at a time (packed fp32)
+                    float2 ls = make_float2(0.f, 0.f);
                     const float mm = m - C::kPScaleLog2;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         float a[4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) a[i] = ex2_approx(fmaf(x[4 * e + i], cs, -mm));
+                        for (int i = 0; i < 4; i += 2) {
+                            const float2 tt = ptx::ffma2(make_float2(x[4 * e + i], x[4 * e + i + 1]),
+                                                         make_float2(cs, cs), make_float2(-mm, -mm));
+                            a[i] = ex2_approx(tt.x);
+                            a[i + 1] = ex2_approx(tt.y);
+                        }
                         // Two terms through f16 pairs: h = a rounded to f16 (relative
                         // error 2^-11); first term = h rounded to E4M3; the remainder
                         // h - first is exact in f16 (a multiple of h's spacing, at most
@@ -651,10 +651,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                         const uint32_t c23 = f16x2_to_e4m3x2(h23);
                         const uint32_t d01 = f16x2_to_e4m3x2(__hsub2(h01, e4m3x2_to_f16x2(c01)));
                         const uint32_t d23 = f16x2_to_e4m3x2(__hsub2(h23, e4m3x2_to_f16x2(c23)));
-                        lsum += (a[0] + a[1]) + (a[2] + a[3]);
+                        ls = ptx::fadd2(ls, ptx::fadd2(make_float2(a[0], a[1]), make_float2(a[2], a[3])));
                         packed[0][e] = c01 | (c23 << 16);
                         packed[1][e] = d01 | (d23 << 16);
                     }
+                    lsum = ls.x + ls.y;
                 };
                 if (!first) exps(m_ref);
                 ok = ptx::mbar_wait_bounded(group_sync, sync_cnt & 1, tmo);

@@ -435,5 +435,54 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(uint32_t M, uint32_t N, u
            | ((M >> 4) << 24);  // M / 16
 }
 
+// Packed fp32 pair arithmetic of sm_100 (one instruction for two lanes of
+// work): d = a * b + c and d = a + b, each half rounded as the scalar form.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// max(a, b, c) in one instruction (sm_100); NaN inputs are ignored as by fmaxf.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// The largest of 64 values: a tree of three-input maxima (32 instructions).
+__device__ __forceinline__ float max64(const float (&x)[64]) {
+    float m1[22];
+#pragma unroll
+    for (int j = 0; j < 21; ++j) m1[j] = fmax3(x[3 * j], x[3 * j + 1], x[3 * j + 2]);
+    m1[21] = x[63];
+    float m2[8];
+#pragma unroll
+    for (int j = 0; j < 7; ++j) m2[j] = fmax3(m1[3 * j], m1[3 * j + 1], m1[3 * j + 2]);
+    m2[7] = m1[21];
+    const float m3a = fmax3(m2[0], m2[1], m2[2]);
+    const float m3b = fmax3(m2[3], m2[4], m2[5]);
+    return fmax3(m3a, m3b, fmaxf(m2[6], m2[7]));
+}
+
 }  // namespace ptx
 }  // namespace mla
