@@ -137,8 +137,8 @@ mla_status launch_pair(const mla_plan& plan, const CUtensorMap& tm_q, const CUte
     return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
-constexpr int kPairFp8NK = 14;  // K chunks of 4 KB
-constexpr int kPairFp8NV = 4;   // V slots of 16 KB (two tiles)
+constexpr int kPairFp8NK = 18;  // K chunks of 4 KB (two tiles)
+constexpr int kPairFp8NV = 3;   // V slots of 16 KB (a tile and a half)
 using PairFp8C = mla::PairFp8Cfg<kPairFp8NK, kPairFp8NV, kPairNS, kPairNP>;
 
 mla_status launch_pair_fp8(const mla_plan& plan, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
