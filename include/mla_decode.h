@@ -345,13 +345,13 @@ mla_status mha_decode_run_phase(const mla_plan* plan, const void* q, const void*
  *   MLA_KERNEL_FP8_PAIR (the default when Sq*H is a multiple of 128): the
  *     codes are the operands of kind::f8f6f4 MMAs on a CTA pair; each q row is
  *     scaled by a power of two and carried as the sum of two E4M3 terms (about
- *     8 significant bits, the precision of a bf16 q), and P (scaled by 2^7) as
+ *     8 significant bits, the precision of a bf16 q), and P (scaled by 2^4) as
  *     the sum of two (about 8 bits, the precision of the bf16 P of the bf16
  *     path).
  *   MLA_KERNEL_FP8_MMA (the default otherwise): the codes are the operands of
  *     kind::f8f6f4 tensor-core MMAs as they are; each q row is scaled by a
  *     power of two and carried as the sum of three E4M3 terms (about 12
- *     significant bits, relative error <= 2^-12), and P (scaled by 2^7) as the
+ *     significant bits, relative error <= 2^-12), and P (scaled by 2^4) as the
  *     sum of two (about 8 bits, the precision of the bf16 P of the bf16 path).
  *   MLA_KERNEL_FP8: every E4M3 value divided by 2^8 is exact in f16, so the
  *     kernel widens the codes to those f16 values in shared memory (integer

@@ -13,13 +13,14 @@
 //      about 12 significant bits.  The three terms are the N columns
 //      [0, G), [G, 2G), [2G, 3G) of one S^T MMA, so every K tile is read
 //      once:  S^T[kv, j] = (sum_k S^T_k[kv, j]) * 2^-e_j.
-//   P: scaled by 2^7 and written as the sum of two E4M3 terms (about 8
+//   P: scaled by 2^4 and written as the sum of two E4M3 terms (about 8
 //      significant bits, the precision of the bf16 P of the other kernels);
 //      the two terms are the N columns [0, G) and [G, 2G) of the PV MMAs,
-//      O^T = O^T_1 + O^T_2.  The reference max is raised whenever a column's
-//      max exceeds it by more than 1 (base 2), so 2^7 p <= 256 stays inside
-//      E4M3 while the weights of far smaller scores keep normal codes (at
-//      scale 1 they would fall into the subnormal range and lose precision).
+//      O^T = O^T_1 + O^T_2.  The reference max is raised only when a column's
+//      max exceeds it by more than 4 (base 2), so 2^4 p <= 256 stays inside
+//      E4M3 while weights down to 2^-10 of the reference keep normal codes
+//      (at scale 1 the smaller ones would fall into the subnormal range and
+//      lose precision; a threshold of 1 with 2^7 p rescaled O far more often).
 //
 // K and V are exact; the errors are the truncation of q (<= 2^-12 relative)
 // and of p (<= 2^-8 relative), and fp32 accumulation.  A host-side emulation
@@ -93,8 +94,9 @@ struct Fp8MmaCfg {
     // kind::f8f6f4 with E4M3 A and B: format codes 0, the same bit layout as f16
     static constexpr uint32_t kIdescS = ptx::make_idesc_f16(128, NS, 0, 0);
     static constexpr uint32_t kIdescPV = ptx::make_idesc_f16(128, NO, 1, 1);
-    static constexpr float kLazy = 1.f;      // rescale threshold (base-2 units): p <= 2
-    static constexpr float kPScaleLog2 = 7.f;  // P is carried as 2^7 p <= 256
+    static constexpr float kLazy = 4.f;      // rescale threshold (base-2 units): p <= 16
+    static constexpr float kPScaleLog2 = 4.f;  // P is carried as 2^4 p <= 256
+    static constexpr float kPScaleInv = 1.f / 16.f;
 };
 
 // D[tmem] (+)= A[smem] . B[smem], both E4M3, K = 32 per instruction.
@@ -569,7 +571,7 @@ __global__ void __launch_bounds__(192, 1)
                     tmax[j + 2] = fmaxf(fmaxf(a.z, b1.z), fmaxf(b2.z, b3.z));
                     tmax[j + 3] = fmaxf(fmaxf(a.w, b1.w), fmaxf(b2.w, b3.w));
                 }
-                // lazy rescale (threshold kLazy, so 2^7 p <= 256 < 448), uniform branch
+                // lazy rescale (threshold kLazy, so 2^4 p <= 256 < 448), uniform branch
                 bool grow = false;
 #pragma unroll
                 for (int j = 0; j < G; ++j) grow |= (tmax[j] > m_ref[j] + C::kLazy);
@@ -606,7 +608,7 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     ptx::tmem_wait_st();
                 }
-                // P terms of this kv row: 2^7 p = t1 + t2 (E4M3), t1 in bytes [0, G), t2 in [G, 2G);
+                // P terms of this kv row: 2^4 p = t1 + t2 (E4M3), t1 in bytes [0, G), t2 in [G, 2G);
                 // P buffer sb was last read by the PV of tile - 2, which the tensor pipe ran
                 // before this tile's S^T
                 uint8_t* p_buf = p_smem + sb * C::kPBytes;
@@ -662,12 +664,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                 for (int jj = 0; jj < G; ++jj)
                     if (jj == j) mj = m_ref[jj];
-                // the sums and O carry the 2^7 of P: l is unscaled here, O in fin
+                // the sums and O carry the 2^4 of P: l is unscaled here, O in fin
                 float lj = (redsum[0 * G + j] + redsum[1 * G + j] + redsum[2 * G + j] + redsum[3 * G + j]) *
-                           0.0078125f;
+                           C::kPScaleInv;
                 float c = 1.f;
                 if (sink_here) c = fold_sink(mj, lj, args.sinks[qr % args.H] * kLog2e);
-                fin[j] = c / lj * args.o_scale * 0.0078125f;
+                fin[j] = c / lj * args.o_scale * C::kPScaleInv;
                 const float lse_nat = (mj + log2f(lj)) * 0.69314718055994530942f;
                 if (pc.slot < 0)
                     args.lse[static_cast<size_t>(pc.b) * args.R + qr] = lse_nat;

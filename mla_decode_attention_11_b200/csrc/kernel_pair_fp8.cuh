@@ -13,13 +13,15 @@
 //      about 8 significant bits (the precision of a bf16 q).  Both terms
 //      multiply the same K chunk into the same S accumulator, so
 //      S = (t1 + t2) K^T and the softmax multiplies each row by 2^-e.
-//   P: carried as 2^7 p, rounded to f16 and written as two E4M3 terms
+//   P: carried as 2^4 p, rounded to f16 and written as two E4M3 terms
 //      t1 = e4m3(h), t2 = e4m3(h - t1) (about 8 significant bits, the
 //      precision of the bf16 P of the other kernels); both multiply the same
-//      V chunk into O.  The row sum adds the fp32 weights 2^7 p, so the
-//      factor 2^7 cancels in O / l; the reference max is raised whenever a row
-//      max exceeds it by more than 1 (base 2), so 2^7 p <= 256 stays inside
-//      E4M3 while small weights keep normal codes.
+//      V chunk into O.  The row sum adds the fp32 weights 2^4 p, so the
+//      factor 2^4 cancels in O / l; the reference max is raised only when a
+//      row max exceeds it by more than 4 (base 2), so 2^4 p <= 256 stays
+//      inside E4M3 while weights down to 2^-10 of the reference keep normal
+//      codes.  (A threshold of 1 with 2^7 p rescaled O several times per
+//      row, each time waiting for the PV in flight.)
 //
 // With K = 32 codes per instruction and two terms, the MMA count and the
 // tensor time per tile are those of the bf16 pair kernel; the cache bytes
@@ -87,8 +89,9 @@ struct PairFp8Cfg {
     // kind::f8f6f4 with E4M3 A and B: format codes 0 (the bit layout of the f16 descriptor)
     static constexpr uint32_t kIdescS = ptx::make_idesc_f16(128, 128, 0, 0);
     static constexpr uint32_t kIdescPV = ptx::make_idesc_f16(128, 256, 0, 1);
-    static constexpr float kLazy = 1.f;        // rescale threshold (base 2): 2^7 p <= 256
-    static constexpr float kPScaleLog2 = 7.f;  // P carried as 2^7 p
+    static constexpr float kLazy = 4.f;        // rescale threshold (base 2): 2^4 p <= 256
+    static constexpr float kPScaleLog2 = 4.f;  // P carried as 2^4 p
+    static constexpr float kPScaleInv = 1.f / 16.f;
     static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -572,7 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             }
             const float row_cs = args.scale_log2 * qscale[r];  // score scale of this row (base 2)
             float m_ref = -INFINITY;  // reference max (base 2) of the row, the same in both of its threads
-            float l_part = 0.f;       // this thread's share of the row sum (of 2^7 p), relative to m_ref
+            float l_part = 0.f;       // this thread's share of the row sum (of 2^4 p), relative to m_ref
             for (int t = pc.tile_lo; t < pc.tile_hi; ++t) {
                 const bool first = (t == pc.tile_lo);
                 int row0 = t * kTileKV;
@@ -615,11 +618,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 float* redmax = red + (tile_cnt & 1) * 128;
                 redmax[L_id] = mloc;
                 ptx::mbar_arrive(group_sync);
-                // 2^7 P[r][64h .. 64h+63] = exp2(x * cs - m_ref + 7) as two E4M3
+                // 2^4 P[r][64h .. 64h+63] = exp2(x * cs - m_ref + 4) as two E4M3
                 // terms.  Past a piece's first tile the reference max is known
                 // before this tile's max, so P is computed at once; it is redone
-                // only when the row max outgrew the reference by more than 1
-                // (2^7 p <= 256).
+                // only when the row max outgrew the reference by more than 4
+                // (2^4 p <= 256).
                 uint32_t packed[2][16];  // term k: 64 codes in 16 words
                 float lsum = 0.f;
                 auto exps = [&](float m) {
@@ -642,9 +645,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                         // half the first term's spacing, so under 8 significant bits);
                         // second term = the remainder rounded to E4M3.  The pair holds a
                         // to about 2^-8 relative (below E4M3's normal range, to its
-                        // subnormal spacing 2^-9: under 2^-16 of the row sum, whose
-                        // largest term is 2^7).  The row sum takes the fp32 weights, as
-                        // in the bf16 kernel.
+                        // subnormal spacing 2^-9: under 2^-13 of the row sum, which
+                        // holds a term of 2^4).  The row sum takes the fp32 weights,
+                        // as in the bf16 kernel.
                         const __half2 h01 = __floats2half2_rn(a[0], a[1]);
                         const __half2 h23 = __floats2half2_rn(a[2], a[3]);
                         const uint32_t c01 = f16x2_to_e4m3x2(h01);
@@ -737,13 +740,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             ok = group_barrier();
             if (!ok) break;
             const int qrow = g * 128 + static_cast<int>(rank) * 64 + r;  // row within the sequence
-            // l and O both carry the factor 2^7 of the P terms
-            float l_row = (l_part + redsum[L_id ^ 64]) * (1.f / 128.f);
+            // l and O both carry the factor 2^4 of the P terms
+            float l_row = (l_part + redsum[L_id ^ 64]) * C::kPScaleInv;
             // a sink applies once per row: to whole sequences here, to cut ones in the combine
             float o_fac = 1.f;
             if (args.sinks != nullptr && pc.slot < 0)
                 o_fac = fold_sink(m_ref, l_row, args.sinks[qrow % args.H] * kLog2e);
-            const float inv_l = o_fac * args.o_scale * (1.f / 128.f) / l_row;
+            const float inv_l = o_fac * args.o_scale * C::kPScaleInv / l_row;
             if (h == 0) {
                 const float lse_nat = (m_ref + log2f(l_row)) * 0.69314718055994530942f;
                 if (pc.slot < 0)
