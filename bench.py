@@ -673,6 +673,7 @@ def run_fp8(args, w: W.Workload):
     flops, nbytes = w.algorithmic_flops(sl), w.algorithmic_bytes_fp8(sl)
     peaks, peak_src = load_peaks()
     cpu_base = None
+    check = None
     if not args.no_cpu_baseline:
         import numpy as np
         import oracle
@@ -680,17 +681,28 @@ def run_fp8(args, w: W.Workload):
         b0 = 0
         rows = np.arange(b0 * R, (b0 + 1) * R, dtype=np.int64)
         t0 = time.perf_counter()
-        oracle.mla_decode_fp8(q, codes, ks, sl, w.scale, row_ids=rows)
+        ro, rl = oracle.mla_decode_fp8(q, codes, ks, sl, w.scale, row_ids=rows)
         dt = time.perf_counter() - t0
+        check = compare_rows(out.reshape(-1, W.D_V)[torch.from_numpy(rows)].cpu().to(torch.float64).numpy(),
+                             lse.reshape(-1)[torch.from_numpy(rows)].cpu().to(torch.float64).numpy(),
+                             np.asarray(ro, dtype=np.float64).reshape(len(rows), W.D_V),
+                             np.asarray(rl, dtype=np.float64).reshape(-1))
         f_cpu = int(sl[b0]) * R * 2 * (W.D_QK + W.D_V)
         cpu_base = {"value": f_cpu / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
                     "sample": f"1 of {w.B} sequences, all {R} query rows, {dt:.1f} s of fp64 CPU work"}
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    # The tensor peak of the kernel's own MMA type: f16 MMAs (the widening
+    # kernel) run at the measured bf16 rate; E4M3 MMAs (kind::f8f6f4) at twice
+    # it (the nominal 4.5 / 2.25 PFLOP/s ratio).  The algorithmic flops are the
+    # definition's: the E4M3 kernels' extra MMAs for the q and P terms are
+    # their own cost, not work of the decode.
+    e4m3_mma = plan.kernel in (M.MLA_KERNEL_FP8_PAIR, M.MLA_KERNEL_FP8_MMA)
+    tensor_peak = peaks["bf16_tflops"] * (2.0 if e4m3_mma else 1.0)
+    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     bound = "hbm" if flops / nbytes < ridge else "tensor"
     if bound == "hbm":
         achieved, peak, unit = nbytes / (main_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
-    else:  # f16 MMAs: the measured bf16 figure (same dense rate)
-        achieved, peak, unit = flops / (main_ms * 1e-3) / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    else:
+        achieved, peak, unit = flops / (main_ms * 1e-3) / 1e12, tensor_peak, "TFLOP/s"
     fp8_kernel_label, fp8_kernel_name, traffic_key = {
         M.MLA_KERNEL_FP8_PAIR: ("FP8 operands on a CTA pair (kind::f8f6f4)", "mla_decode_pair_fp8_kernel",
                                 w.name + "_fp8"),
@@ -719,15 +731,25 @@ def run_fp8(args, w: W.Workload):
                      "kernel": fp8_kernel_name, "kernel_ms": main_ms,
                      "combine_ms": comb_ms, "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
                      "hbm_frac": nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "tensor_frac": flops / (main_ms * 1e-3) / 1e12 / tensor_peak,
+                     "tensor_peak_tflops": tensor_peak,
+                     "tensor_peak_note": ("E4M3 MMAs: twice the bf16 figure (nominal 4.5 / 2.25 PFLOP/s)"
+                                          if e4m3_mma else "f16 MMAs: the bf16 figure"),
                      "step_roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
-                                               flops / (peaks["bf16_tflops"] * 1e12)) * 1e3 / t_ms},
+                                               flops / (tensor_peak * 1e12)) * 1e3 / t_ms},
         "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": q.numel() * 2 + codes.numel() + sl.numel() * 4,
                 "d2h_bytes_per_step": out.numel() * 2 + lse.numel() * 4, "ms_per_step": e2e_ms},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu_base,
+        "output_check": check,
     }
+    frac = achieved / peak
+    if not (0.0 < frac <= MAX_PLAUSIBLE_FRAC):
+        refuse(line, f"roofline fraction {frac:.3f} is outside (0, {MAX_PLAUSIBLE_FRAC}]")
+    if check is not None and check.get("ok") is False:
+        refuse(line, "the timed run's outputs do not match the oracle")
     print(json.dumps(line), flush=True)
 
 
