@@ -456,16 +456,23 @@ __global__ void __launch_bounds__(192, 1)
                 if (!ok) break;
             }
             {
+                // this thread's 16-byte units qpart, qpart + kThrPerRow, ... of the row,
+                // loaded at once (one round trip to memory)
+                constexpr int kQUnits = kDqk / 8 / kThrPerRow;
+                static_assert(kQUnits * kThrPerRow * 8 == kDqk, "q units per thread");
                 const uint4* qrow =
                     reinterpret_cast<const uint4*>(args.q + (static_cast<size_t>(pc.b) * args.R + g * G + qj) * kDqk);
-                float amax = 0.f;
-                for (int sg = qpart; sg < kDqk / 8; sg += kThrPerRow) {
-                    const uint4 v = __ldg(qrow + sg);
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                uint4 qv[kQUnits];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-                        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                for (int i = 0; i < kQUnits; ++i) qv[i] = __ldg(qrow + qpart + i * kThrPerRow);
+                float amax = 0.f;
+#pragma unroll
+                for (int i = 0; i < kQUnits; ++i) {
+                    const uint32_t w[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+                        amax = ptx::fmax3(amax, fabsf(f.x), fabsf(f.y));
                     }
                 }
 #pragma unroll
@@ -473,9 +480,10 @@ __global__ void __launch_bounds__(192, 1)
                 const int e = q_row_exponent(amax);
                 if (qpart == 0) qscale[qj] = ldexpf(args.scale_log2, -e);
                 const float up = ldexpf(1.f, e);
-                for (int sg = qpart; sg < kDqk / 8; sg += kThrPerRow) {
-                    const uint4 v = __ldg(qrow + sg);
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < kQUnits; ++i) {
+                    const int sg = qpart + i * kThrPerRow;
+                    const uint32_t w[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
                     float x[8];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {

@@ -500,25 +500,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         };
         Piece pc;
         while (ok && walker.next(pc)) {
-            // ---------------- the piece's Q as two E4M3 terms.  Thread (r, h) writes
-            // chunks [0, 5) (h = 0) or [5, 9) (h = 1) of row r, after the previous
-            // piece's last QK^T has read the old terms
+            // ---------------- the piece's Q as two E4M3 terms.  Thread (r, h) takes
+            // 16-byte units [36h, 36h + 36) of row r in three batches of 12, each
+            // batch's loads issued together: the row max over the three, then the
+            // terms (the last batch still in registers, the first two reloaded),
+            // written after the previous piece's last QK^T has read the old ones
             {
                 if (piece_cnt > 0) {
                     ok = ptx::mbar_wait_bounded(q_empty, (piece_cnt - 1) & 1, tmo);
                     if (!ok) break;
                 }
-                const int c_lo = h ? 5 : 0, c_hi = h ? kNumChunks : 5;
+                constexpr int kQUnits = kDqk / 8 / 2;  // 16-byte units (8 bf16) per thread
+                constexpr int kQBatch = 12;
+                constexpr int kQBatches = kQUnits / kQBatch;
+                static_assert(kQBatches * kQBatch == kQUnits, "q batches");
                 const uint4* qsrc = reinterpret_cast<const uint4*>(
-                    args.q + (static_cast<size_t>(pc.b) * args.R + g * 128 + static_cast<int>(rank) * 64 + r) * kDqk);
+                    args.q + (static_cast<size_t>(pc.b) * args.R + g * 128 + static_cast<int>(rank) * 64 + r) * kDqk) +
+                    kQUnits * h;
+                uint4 qv[kQBatch];
                 float amax = 0.f;
-                for (int sg = c_lo * 8; sg < c_hi * 8; ++sg) {  // 8 bf16 per 16 bytes
-                    const uint4 v = __ldg(qsrc + sg);
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-                        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+                for (int bt = 0; bt < kQBatches; ++bt) {
+#pragma unroll
+                    for (int i = 0; i < kQBatch; ++i) qv[i] = __ldg(qsrc + bt * kQBatch + i);
+#pragma unroll
+                    for (int i = 0; i < kQBatch; ++i) {
+                        const uint32_t w[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+                            amax = ptx::fmax3(amax, fabsf(f.x), fabsf(f.y));
+                        }
                     }
                 }
                 qamax[L_id] = amax;
@@ -528,41 +540,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
                 const int e = q_row_exponent(amax);
                 if (h == 0) qscale[r] = ldexpf(1.f, -e);
                 const float up = ldexpf(1.f, e);
-                for (int sg = c_lo * 8; sg < c_hi * 8; ++sg) {
-                    const uint4 v = __ldg(qsrc + sg);
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                    float x[8];
+#pragma unroll 1
+                for (int bt = kQBatches - 1; bt >= 0; --bt) {
+                    if (bt != kQBatches - 1) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-                        x[2 * i] = f.x * up;
-                        x[2 * i + 1] = f.y * up;
+                        for (int i = 0; i < kQBatch; ++i) qv[i] = __ldg(qsrc + bt * kQBatch + i);
                     }
-                    uint32_t tw[2][2];  // term k: 8 codes in two words
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
+                    for (int i = 0; i < kQBatch; ++i) {
+                        const uint32_t w[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+                        float x[8];
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const uint32_t c01 = f32x2_to_e4m3x2(x[4 * hh], x[4 * hh + 1]);
-                            const uint32_t c23 = f32x2_to_e4m3x2(x[4 * hh + 2], x[4 * hh + 3]);
-                            tw[k][hh] = c01 | (c23 << 16);
-                            const float2 v01 = e4m3x2_to_f32x2(c01);
-                            const float2 v23 = e4m3x2_to_f32x2(c23);
-                            x[4 * hh] -= v01.x;
-                            x[4 * hh + 1] -= v01.y;
-                            x[4 * hh + 2] -= v23.x;
-                            x[4 * hh + 3] -= v23.y;
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+                            x[2 * j] = f.x * up;
+                            x[2 * j + 1] = f.y * up;
                         }
-                    }
-                    // codes d0 .. d0+7 of chunk d0 / 64: half of one 16-byte unit of row r
-                    const int d0 = sg * 8;
-                    const uint32_t u = static_cast<uint32_t>((d0 % kChunk) / 16);
-                    const uint32_t half8 = static_cast<uint32_t>((d0 % 16) / 8) * 8;
+                        uint32_t tw[2][2];  // term k: 8 codes in two words
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        uint8_t* chunk = q_smem + (k * kNumChunks + d0 / kChunk) * C::kQChunk;
-                        *reinterpret_cast<uint2*>(chunk + swz_offset(static_cast<uint32_t>(r), u, 64) + half8) =
-                            make_uint2(tw[k][0], tw[k][1]);
+                        for (int k = 0; k < 2; ++k) {
+#pragma unroll
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const uint32_t c01 = f32x2_to_e4m3x2(x[4 * hh], x[4 * hh + 1]);
+                                const uint32_t c23 = f32x2_to_e4m3x2(x[4 * hh + 2], x[4 * hh + 3]);
+                                tw[k][hh] = c01 | (c23 << 16);
+                                const float2 v01 = e4m3x2_to_f32x2(c01);
+                                const float2 v23 = e4m3x2_to_f32x2(c23);
+                                x[4 * hh] -= v01.x;
+                                x[4 * hh + 1] -= v01.y;
+                                x[4 * hh + 2] -= v23.x;
+                                x[4 * hh + 3] -= v23.y;
+                            }
+                        }
+                        // codes d0 .. d0+7 of chunk d0 / 64: half of one 16-byte unit of row r
+                        const int d0 = (kQUnits * h + bt * kQBatch + i) * 8;
+                        const uint32_t u = static_cast<uint32_t>((d0 % kChunk) / 16);
+                        const uint32_t half8 = static_cast<uint32_t>((d0 % 16) / 8) * 8;
+#pragma unroll
+                        for (int k = 0; k < 2; ++k) {
+                            uint8_t* chunk = q_smem + (k * kNumChunks + d0 / kChunk) * C::kQChunk;
+                            *reinterpret_cast<uint2*>(chunk + swz_offset(static_cast<uint32_t>(r), u, 64) + half8) =
+                                make_uint2(tw[k][0], tw[k][1]);
+                        }
                     }
                 }
                 ptx::fence_proxy_async_smem();
