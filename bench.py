@@ -621,6 +621,14 @@ def run_fp8(args, w: W.Workload):
             step()
     M.mla_decode_check(plan, ws, stream=stream)
 
+    # As for the bf16 cache: a cache smaller than twice L2 gets an L2 flush
+    # before every timed decode, each decode timed by its own events; a larger
+    # one streams as it is, the decodes replayed as one CUDA graph.
+    l2_bytes = float(torch.cuda.get_device_properties(dev).L2_cache_size)
+    cache_bytes = float(codes.numel())
+    flush_buf = torch.empty(int(2 * l2_bytes), dtype=torch.uint8, device=dev) \
+        if needs_flush(cache_bytes, l2_bytes) else None
+
     def capture(fn, n):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
@@ -629,27 +637,51 @@ def run_fp8(args, w: W.Workload):
                     fn()
         return g
 
-    def replay_ms(g, n):
+    def timed_ms(fn, n):
+        if flush_buf is not None:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            with torch.cuda.stream(stream):
+                torch.cuda._sleep(int(20e6 + 2e6 * n))
+                for i in range(n):
+                    flush_buf.fill_(i & 0xFF)
+                    evs[i][0].record(stream)
+                    fn()
+                    evs[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            return sum(a.elapsed_time(b) for a, b in evs) / n
+        g = capture(fn, n)
+        torch.cuda.synchronize(dev)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             a.record(stream)
             g.replay()
             b.record(stream)
         torch.cuda.synchronize(dev)
+        del g
         return a.elapsed_time(b) / n
 
-    g_steps = capture(step, args.steps)
-    torch.cuda.synchronize(dev)
+    if flush_buf is None:
+        g_steps = capture(step, args.steps)
+        torch.cuda.synchronize(dev)
     clocks = ClockSampler(0)
     clocks.start()
-    t_ms = replay_ms(g_steps, args.steps)
+    if flush_buf is None:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g_steps.replay()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        t_ms = a.elapsed_time(b) / args.steps
+        del g_steps
+    else:
+        t_ms = timed_ms(step, args.steps)
     clk = clocks.stop()
-    del g_steps
     n_brk = max(3, min(args.steps, 50))
-    main_ms = replay_ms(capture(lambda: M.mla_decode_run_fp8_phase(plan, qd, cd, ks, sld, w.scale, out, lse, ws, 1,
-                                                                   stream=stream), n_brk), n_brk)
-    comb_ms = replay_ms(capture(lambda: M.mla_decode_run_fp8_phase(plan, qd, cd, ks, sld, w.scale, out, lse, ws, 2,
-                                                                   stream=stream), n_brk), n_brk)
+    main_ms = timed_ms(lambda: M.mla_decode_run_fp8_phase(plan, qd, cd, ks, sld, w.scale, out, lse, ws, 1,
+                                                          stream=stream), n_brk)
+    comb_ms = timed_ms(lambda: M.mla_decode_run_fp8_phase(plan, qd, cd, ks, sld, w.scale, out, lse, ws, 2,
+                                                          stream=stream), n_brk)
     M.mla_decode_check(plan, ws, stream=stream)
     # end to end: host buffers in, host buffers out, copies inside the timed region
     qh, ch, slh = q.pin_memory(), codes.pin_memory(), sl.pin_memory()
@@ -723,7 +755,7 @@ def run_fp8(args, w: W.Workload):
                    "global_batch": w.B, "seq_len": w.L, "parallelism": "single GPU",
                    "kernel": fp8_kernel_label,
                    "group_rows": plan.group_rows, "partitions": plan.num_partitions,
-                   "l2": l2_note(codes.numel())},
+                   "l2": flush_note(cache_bytes, l2_bytes) if flush_buf is not None else l2_note(cache_bytes)},
         "hbm_gbs": nbytes / (t_ms * 1e-3) / 1e9,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
