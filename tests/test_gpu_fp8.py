@@ -170,6 +170,26 @@ def test_fp8_large_scale_and_rescale(cuda_device, kernel):
 
 
 @pytest.mark.parametrize("kernel", FP8_KERNELS)
+def test_fp8_rising_scores_force_rescale(cuda_device, kernel):
+    """Keys whose scores rise along the sequence by ~13.5 (log2 units) per
+    128-key tile: every tile outgrows the reference max by more than any lazy
+    threshold, so the FP8 kernels rescale O on every tile."""
+    H = 128 if kernel == M.MLA_KERNEL_FP8_PAIR else 16
+    w = W.custom(B=1, Sq=1, H=H, L=1024, seed=73)
+    q, kv, sl = W.generate(w)
+    # last rope column: q = 1, key = a ramp of dequantised values 0 .. 1792
+    # (codes 0 .. 448 at kv_scale 4), the other values N(0, 1) as codes of kv / 4
+    q[..., 575] = 1.0
+    ks = 4.0
+    vals = kv.float() / ks
+    vals[0, :, 575] = torch.linspace(0, 448, 1024)
+    codes = vals.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    out, lse, _ = gpu_decode_fp8(q, codes, ks, sl, w.scale, kernel=kernel)
+    ro, rl = oracle.mla_decode_fp8(q, codes, ks, sl, w.scale)
+    assert_parity(out, lse, ro, rl, f"fp8 ramp H{H}", out_max_abs=OUT_MAX_ABS * max(1.0, float(np.abs(ro).max())))
+
+
+@pytest.mark.parametrize("kernel", FP8_KERNELS)
 def test_fp8_deterministic_and_split_invariant(cuda_device, kernel):
     w = W.custom(B=4, Sq=1, H=128, L=2500, L_lo=100, seed=195)
     q, codes, ks, sl = W.generate_fp8(w)
