@@ -95,6 +95,24 @@ def compare_rows(out_rows, lse_rows, ref_out, ref_lse) -> dict:
             "tolerance": "max-abs 2e-2, rel-L2 5e-3, lse 1e-3", "ok": ok}
 
 
+def mma_tensor_peak(peaks: dict, e4m3_mma: bool) -> float:
+    """Dense tensor peak (TFLOP/s) of a kernel's own MMA type: bf16 and f16
+    MMAs run at the measured bf16 rate, E4M3 MMAs (kind::f8f6f4) at twice it
+    (the nominal 4.5 / 2.25 PFLOP/s ratio).  The algorithmic flops stay the
+    definition's: the E4M3 kernels' extra MMAs for their q and P terms are
+    their own cost, not work of the decode."""
+    return peaks["bf16_tflops"] * (2.0 if e4m3_mma else 1.0)
+
+
+def roofline_point(flops: float, nbytes: float, kernel_ms: float, hbm_gbs: float, tensor_tflops: float):
+    """(bound, achieved, peak, unit) of one kernel launch: HBM-bound when the
+    arithmetic intensity is below the ridge of the two peaks, else tensor-bound."""
+    ridge = tensor_tflops * 1e12 / (hbm_gbs * 1e9)
+    if flops / nbytes < ridge:
+        return "hbm", nbytes / (kernel_ms * 1e-3) / 1e9, hbm_gbs, "GB/s"
+    return "tensor", flops / (kernel_ms * 1e-3) / 1e12, tensor_tflops, "TFLOP/s"
+
+
 def refuse(line: dict, why: str) -> None:
     """A number that cannot be right is not printed as a result."""
     sys.stderr.write("bench.py: refusing to report this measurement: %s\n%s\n" % (why, json.dumps(line)))
@@ -400,19 +418,9 @@ def run_ours(args, w: W.Workload):
     peaks, peak_src = load_peaks()
     value = whole_job_rate(world, flops, t_ms) / 1e12
     hbm_gbs = whole_job_rate(world, nbytes, t_ms) / 1e9
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    ai = flops / nbytes
-    bound = "hbm" if ai < ridge else "tensor"
-    if bound == "hbm":
-        achieved = nbytes / (main_avg * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        spec = SPEC_PEAKS["hbm_gbs"]
-        unit = "GB/s"
-    else:
-        achieved = flops / (main_avg * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        spec = SPEC_PEAKS["bf16_tflops"]
-        unit = "TFLOP/s"
+    bound, achieved, peak, unit = roofline_point(flops, nbytes, main_avg, peaks["hbm_gbs"],
+                                                 mma_tensor_peak(peaks, e4m3_mma=False))
+    spec = SPEC_PEAKS["hbm_gbs"] if bound == "hbm" else SPEC_PEAKS["bf16_tflops"]
     roof_time_ms = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e3
     # the record was taken with the default plan; a batch-invariant plan moves other bytes
     traffic, traffic_note = load_traffic(w.name) if not plan.split_tiles else (None, None)
@@ -722,19 +730,9 @@ def run_fp8(args, w: W.Workload):
         f_cpu = int(sl[b0]) * R * 2 * (W.D_QK + W.D_V)
         cpu_base = {"value": f_cpu / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.max_threads(), "kind": "oracle",
                     "sample": f"1 of {w.B} sequences, all {R} query rows, {dt:.1f} s of fp64 CPU work"}
-    # The tensor peak of the kernel's own MMA type: f16 MMAs (the widening
-    # kernel) run at the measured bf16 rate; E4M3 MMAs (kind::f8f6f4) at twice
-    # it (the nominal 4.5 / 2.25 PFLOP/s ratio).  The algorithmic flops are the
-    # definition's: the E4M3 kernels' extra MMAs for the q and P terms are
-    # their own cost, not work of the decode.
     e4m3_mma = plan.kernel in (M.MLA_KERNEL_FP8_PAIR, M.MLA_KERNEL_FP8_MMA)
-    tensor_peak = peaks["bf16_tflops"] * (2.0 if e4m3_mma else 1.0)
-    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    bound = "hbm" if flops / nbytes < ridge else "tensor"
-    if bound == "hbm":
-        achieved, peak, unit = nbytes / (main_ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s"
-    else:
-        achieved, peak, unit = flops / (main_ms * 1e-3) / 1e12, tensor_peak, "TFLOP/s"
+    tensor_peak = mma_tensor_peak(peaks, e4m3_mma)
+    bound, achieved, peak, unit = roofline_point(flops, nbytes, main_ms, peaks["hbm_gbs"], tensor_peak)
     fp8_kernel_label, fp8_kernel_name, traffic_key = {
         M.MLA_KERNEL_FP8_PAIR: ("FP8 operands on a CTA pair (kind::f8f6f4)", "mla_decode_pair_fp8_kernel",
                                 w.name + "_fp8"),
